@@ -1,0 +1,406 @@
+"""Benchmark: CommVQ decode attention, KV tokens/s per layer on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--form gqa|table]
+    python bench.py --impl reference ...     # the float64 CPU oracle, timed on host cores
+
+A step is one decode-attention pass over one layer of the workload: every query head
+of every sequence against its whole cached code stream (decode + combine; the table
+form adds the query-table build).  Inputs are resident in HBM before timing; 8
+independent layer-sized input sets rotate from step to step so no step finds the
+previous one's codes in L2 (8 x 36 MB > 126 MB L2 for the 128K layer).
+
+Printed: one JSON line (rank 0) with the metric, the decode kernel's roofline
+fraction (FP32 ALU bound), an end-to-end figure through host buffers, the clocks
+sampled during the timed region and a CPU baseline (the oracle on a bounded sample).
+Under torchrun each rank decodes its own copy of the workload (weak scaling; the
+path shards by sequence and KV head and needs no collective); the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama8b_layer_T131072_R1"
+METRIC = "CommVQ decode attn: KV tokens/s per layer; code HBM GB/s vs B200 peak"
+FP32_LANES_PER_SM = 128
+SM_COUNT_B200 = 148
+N_INPUT_SETS = 8
+
+
+def algorithmic_flops(w: workloads.Workload, total_tokens: int) -> float:
+    """Algorithmic FP32 work of one layer step (per token per query head: 64 pairs x
+    (2 mul + 2 add) = 256, plus 128 (R - 1) adds to sum the rounds, plus 16 R bin adds;
+    exp and sin/cos are counted on the SFU, not here)."""
+    per_tok_head = 256 + 128 * (w.R - 1) + 16 * w.R
+    return float(total_tokens) * w.n_q_heads * per_tok_head
+
+
+def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
+    """Bytes that must come from HBM per layer step: key + value codes of every token of
+    every KV head, plus the key and value codebooks of every KV head."""
+    codes = float(total_tokens) * w.n_kv_heads * 32 * w.R
+    cbs = 2.0 * w.n_kv_heads * 16 * w.R * 256 * 8 * 4
+    return codes + cbs
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+def oracle_sample(w: workloads.Workload, budget_s: float = 12.0, layer: int = 0):
+    """Time the oracle, as it stands, on a sample of (sequence, query head) pairs of
+    one layer until about `budget_s` seconds of CPU work; return tokens/s per layer
+    scaled to the whole layer, the thread count and what the sample was."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import cvq_oracle as O
+
+    d = workloads.generate(w, layer=layer)
+    lens = d["seq_lens"]
+    total_tokens = int(lens.sum())
+    heads = [(b, h) for b in range(w.batch) for h in range(w.n_q_heads)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(heads)
+    done_tokens = 0
+    n = 0
+    t0 = time.perf_counter()
+    with threadpool_limits(1):
+        for b, hq in heads:
+            h = O.kv_head_of(hq, w.n_q_heads, w.n_kv_heads)
+            O.attend_head(d["q"][b, hq], d["key_cb"][h], d["val_cb"][h], d["key_codes"][b, h],
+                          d["val_codes"][b, h], int(lens[b]), d["rope_base"])
+            done_tokens += int(lens[b])
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+    el = time.perf_counter() - t0
+    # one layer = every query head over its sequence: scale the token-heads done
+    layer_time = el * (total_tokens * w.n_q_heads) / max(done_tokens, 1)
+    return {"value": total_tokens / layer_time, "unit": "KV tokens/s per layer", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n} of {len(heads)} (sequence, query head) pairs of layer {layer} "
+                      f"({done_tokens} token-heads, {el:.1f} s), scaled to the full layer",
+            "seconds_per_layer": layer_time}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_attention_cvq_b200 as cvq
+    from compressed_attention_cvq_b200 import _binding as _b
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = workloads.WORKLOADS[args.workload]
+    n_sets = N_INPUT_SETS
+    sets = []
+    for i in range(n_sets):
+        d = workloads.generate(w, layer=i)
+        if d["q_dtype"] == "bf16":
+            q = torch.from_numpy(d["q_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+        else:
+            q = torch.from_numpy(d["q"]).to(dev)
+        sets.append(dict(q=q, key_cb=torch.from_numpy(d["key_cb"]).to(dev),
+                         val_cb=torch.from_numpy(d["val_cb"]).to(dev),
+                         key_codes=torch.from_numpy(d["key_codes"]).to(dev),
+                         val_codes=torch.from_numpy(d["val_codes"]).to(dev),
+                         seq_lens=torch.from_numpy(d["seq_lens"]).to(dev),
+                         host=d))
+    total_tokens = int(sets[0]["host"]["seq_lens"].sum())
+    shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base)
+    S = args.splits or cvq.suggest_splits(shape)
+    parts = cvq.partials_alloc(shape, S, dev)
+    out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
+    ptab = (torch.empty((w.batch, w.n_q_heads, 16, w.R, 256, 4, 2), dtype=torch.float32, device=dev)
+            if args.form == "table" else None)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 3 if args.form == "table" else 2
+
+    def step(i, ev=None):
+        s = sets[i % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        if args.form == "table":
+            cvq.qtable(shape, s["q"], s["key_cb"], ptable=ptab)
+            cvq.decode_attn(shape, ptab, s["key_codes"], s["val_codes"], s["seq_lens"], s["val_cb"],
+                            S, partials=parts)
+        else:
+            cvq.decode_attn_gqa(shape, s["q"], s["key_cb"], s["key_codes"], s["val_codes"],
+                                s["seq_lens"], s["val_cb"], S, partials=parts)
+        if ev is not None:
+            ev[1].record(stream)
+        cvq.combine(shape, S, *parts, out=out, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)   # let the sampler start
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+    ms_per_step = total_ms_max / args.steps
+
+    # end to end through the public API: pinned host inputs -> device -> decode -> host
+    h = sets[0]["host"]
+    if h["q_dtype"] == "bf16":
+        hq = torch.from_numpy(h["q_bits"].view(np.int16)).view(torch.bfloat16)
+    else:
+        hq = torch.from_numpy(h["q"])
+    host_in = dict(q=hq.pin_memory(), key_cb=torch.from_numpy(h["key_cb"]).pin_memory(),
+                   val_cb=torch.from_numpy(h["val_cb"]).pin_memory(),
+                   key_codes=torch.from_numpy(h["key_codes"]).pin_memory(),
+                   val_codes=torch.from_numpy(h["val_codes"]).pin_memory(),
+                   seq_lens=torch.from_numpy(h["seq_lens"]).pin_memory())
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    host_out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory()
+    host_lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+
+    def e2e_step():
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        o, l = cvq.attend(dev_in["q"], dev_in["key_cb"], dev_in["val_cb"], dev_in["key_codes"],
+                          dev_in["val_codes"], dev_in["seq_lens"], w.rope_base, n_splits=S,
+                          form=args.form)
+        host_out.copy_(o, non_blocking=True)
+        host_lse.copy_(l, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    e_start.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / n_e2e
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    result = None
+    if rank == 0:
+        pk, pk_src = peaks()
+        dec_mean_ms = statistics.mean(dec_ms)
+        sm_max = pk.get("sm_max_mhz", 1965.0) or 1965.0
+        fp32_peak_tflops = SM_COUNT_B200 * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+        flops = algorithmic_flops(w, total_tokens)
+        achieved_tflops = flops / (dec_mean_ms * 1e-3) / 1e12
+        bytes_ = code_bytes(w, total_tokens)
+        value = world * total_tokens / (ms_per_step * 1e-3)
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "KV tokens/s per layer",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded codebooks, codes and queries; no trained weights)",
+            "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R,
+                       "q_dtype": w.q_dtype, "form": args.form, "n_splits": S,
+                       "tokens_per_layer": total_tokens,
+                       "l2": f"{N_INPUT_SETS} rotating layer input sets of "
+                             f"{code_bytes(w, total_tokens) / 1e6:.0f} MB (> 126 MB L2 in total)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "decode_ms": dec_mean_ms,
+            "code_hbm_gbs": bytes_ / (dec_mean_ms * 1e-3) / 1e9,
+            "code_hbm_frac": bytes_ / (dec_mean_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "roofline": {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak_tflops,
+                         "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
+                         "traffic": None,
+                         "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {sm_max:.0f} MHz "
+                                        f"(unit counts and max clock; HBM peak {pk_src})"},
+            "e2e": {"value": world * total_tokens / (e2e_ms * 1e-3), "unit": "KV tokens/s per layer",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * launches_per_step,
+            "clocks": clk.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    w = workloads.WORKLOADS[args.workload]
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, budget_s=min(per_step, 5.0))
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for i in range(args.steps):
+        last = oracle_sample(w, budget_s=per_step, layer=0)
+        vals.append(last["value"])
+    el = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    total_tokens = int(workloads.make_seq_lens(w).sum())
+    return {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "KV tokens/s per layer",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_tokens / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R, "q_dtype": w.q_dtype},
+        "cpu_baseline": {"value": value, "unit": "KV tokens/s per layer", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {last['sample']}"},
+        "e2e": {"value": value, "unit": "KV tokens/s per layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": el,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--form", choices=["gqa", "table"], default="gqa")
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    res = run_gpu(args)
+    if res is not None:
+        if not args.no_cpu_baseline and res["n_gpus"] == 1:
+            cb = oracle_sample(workloads.WORKLOADS[args.workload])
+            res["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,174 @@
+"""CommVQ decode attention on B200: Python binding of libcvq.
+
+The three calls of the library, one-to-one with include/cvq.h:
+
+  qtable(shape, q, key_cb)                       -> P table      (cvq_qtable)
+  decode_attn(shape, ptable, codes..., n_splits) -> partials     (cvq_decode_attn)
+  decode_attn_gqa(shape, q, key_cb, codes...)    -> partials     (cvq_decode_attn_gqa)
+  combine(shape, partials)                       -> (out, lse)   (cvq_combine)
+
+plus attend(), which allocates the partial states with torch and runs the calls in
+order.  Tensors are torch CUDA tensors in the layouts documented in cvq.h; work is
+enqueued on torch's current CUDA stream.  torch provides device memory and streams
+only: every arithmetic step runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _binding as _b
+from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa: F401
+
+__all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
+           "attend", "split_tokens", "suggest_splits", "partials_alloc", "CvqError"]
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require(t, name, dtype=None, device=True):
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _q_dtype(q):
+    if q.dtype == torch.float32:
+        return CVQ_F32
+    if q.dtype == torch.bfloat16:
+        return CVQ_BF16
+    raise ValueError(f"q must be float32 or bfloat16, got {q.dtype}")
+
+
+def _head_stride(cb, kind):
+    """Head stride in floats of a codebook tensor.  With a leading KV-head dim
+    (key [Hkv, 16, R, 256, 4, 2], value [Hkv, 16, R, 256, 8]) it is one head's size;
+    without it (key [16, R, 256, 4, 2], value [16, R, 256, 8]) the codebook is shared
+    by every KV head and the stride is 0."""
+    per_head_dims = 6 if kind == "key" else 5
+    if cb.dim() == per_head_dims:
+        return cb.numel() // cb.shape[0]
+    if cb.dim() == per_head_dims - 1:
+        return 0
+    raise ValueError(f"{kind} codebook has {cb.dim()} dims")
+
+
+def shape_of(q, key_codes, rope_base=500000.0):
+    """cvq_shape from q [B, Hq, 128] and key_codes [B, Hkv, T_cap, R, 16]."""
+    B, Hq, D = q.shape
+    _, Hkv, T, R, _ = key_codes.shape
+    return make_shape(B, Hq, Hkv, R, T, rope_base, D)
+
+
+def split_tokens(shape, n_splits):
+    return _b.lib.cvq_split_tokens(ctypes.byref(shape), n_splits)
+
+
+def suggest_splits(shape, sm_count=None):
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return _b.lib.cvq_suggest_splits(ctypes.byref(shape), sm_count)
+
+
+def qtable(shape, q, key_cb, ptable=None, stream=None):
+    _require(q, "q", (torch.float32, torch.bfloat16))
+    _require(key_cb, "key_cb", torch.float32)
+    if ptable is None:
+        ptable = torch.empty((shape.batch, shape.n_q_heads, 16, shape.R, 256, 4, 2),
+                             dtype=torch.float32, device=q.device)
+    _require(ptable, "ptable", torch.float32)
+    st = _b.lib.cvq_qtable(ctypes.byref(shape), _ptr(q), _q_dtype(q), _ptr(key_cb),
+                           _head_stride(key_cb, "key"), _ptr(ptable),
+                           _stream(stream))
+    _b.check(st, "cvq_qtable")
+    return ptable
+
+
+def partials_alloc(shape, n_splits, device):
+    B, Hq = shape.batch, shape.n_q_heads
+    part_o = torch.empty((B, Hq, n_splits, 128), dtype=torch.float32, device=device)
+    part_m = torch.empty((B, Hq, n_splits), dtype=torch.float32, device=device)
+    part_l = torch.empty((B, Hq, n_splits), dtype=torch.float32, device=device)
+    return part_o, part_m, part_l
+
+
+def _codes_check(key_codes, val_codes, seq_lens, val_cb):
+    _require(key_codes, "key_codes", torch.uint8)
+    _require(val_codes, "val_codes", torch.uint8)
+    _require(seq_lens, "seq_lens", torch.int32)
+    _require(val_cb, "val_cb", torch.float32)
+
+
+def decode_attn(shape, ptable, key_codes, val_codes, seq_lens, val_cb, n_splits, partials=None,
+                stream=None):
+    """Table form: gathers from the P table of cvq_qtable."""
+    _require(ptable, "ptable", torch.float32)
+    _codes_check(key_codes, val_codes, seq_lens, val_cb)
+    part_o, part_m, part_l = partials or partials_alloc(shape, n_splits, key_codes.device)
+    st = _b.lib.cvq_decode_attn(ctypes.byref(shape), _ptr(ptable), _ptr(key_codes),
+                                _ptr(val_codes), _ptr(seq_lens), _ptr(val_cb),
+                                _head_stride(val_cb, "val"), n_splits,
+                                _ptr(part_o), _ptr(part_m), _ptr(part_l), _stream(stream))
+    _b.check(st, "cvq_decode_attn")
+    return part_o, part_m, part_l
+
+
+def decode_attn_gqa(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
+                    partials=None, stream=None):
+    """GQA form: one codeword gather + rotation per token, shared by the query heads of
+    a KV head."""
+    _require(q, "q", (torch.float32, torch.bfloat16))
+    _require(key_cb, "key_cb", torch.float32)
+    _codes_check(key_codes, val_codes, seq_lens, val_cb)
+    part_o, part_m, part_l = partials or partials_alloc(shape, n_splits, key_codes.device)
+    st = _b.lib.cvq_decode_attn_gqa(ctypes.byref(shape), _ptr(q), _q_dtype(q), _ptr(key_cb),
+                                    _head_stride(key_cb, "key"),
+                                    _ptr(key_codes), _ptr(val_codes), _ptr(seq_lens), _ptr(val_cb),
+                                    _head_stride(val_cb, "val"), n_splits,
+                                    _ptr(part_o), _ptr(part_m), _ptr(part_l), _stream(stream))
+    _b.check(st, "cvq_decode_attn_gqa")
+    return part_o, part_m, part_l
+
+
+def combine(shape, n_splits, part_o, part_m, part_l, out=None, lse=None, stream=None):
+    if out is None:
+        out = torch.empty((shape.batch, shape.n_q_heads, 128), dtype=torch.float32,
+                          device=part_o.device)
+    if lse is None:
+        lse = torch.empty((shape.batch, shape.n_q_heads), dtype=torch.float32, device=part_o.device)
+    st = _b.lib.cvq_combine(ctypes.byref(shape), n_splits, _ptr(part_o), _ptr(part_m),
+                            _ptr(part_l), _ptr(out), _ptr(lse), _stream(stream))
+    _b.check(st, "cvq_combine")
+    return out, lse
+
+
+def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0, n_splits=None,
+           form="gqa", stream=None):
+    """One decode step: (out [B, Hq, 128], lse [B, Hq]) in fp32.
+
+    form="gqa":   cvq_decode_attn_gqa + cvq_combine
+    form="table": cvq_qtable + cvq_decode_attn + cvq_combine
+    """
+    shape = shape_of(q, key_codes, rope_base)
+    if n_splits is None:
+        n_splits = suggest_splits(shape)
+    if form == "table":
+        P = qtable(shape, q, key_cb, stream=stream)
+        parts = decode_attn(shape, P, key_codes, val_codes, seq_lens, val_cb, n_splits, stream=stream)
+    elif form == "gqa":
+        parts = decode_attn_gqa(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
+                                stream=stream)
+    else:
+        raise ValueError(form)
+    return combine(shape, n_splits, *parts, stream=stream)

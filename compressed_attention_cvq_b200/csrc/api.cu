@@ -1,0 +1,224 @@
+// libcvq C ABI: argument validation on the host, then kernel launches.  Nothing is
+// allocated and no state is kept; every error is returned as a cvq_status before any
+// launch.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+using namespace cvq;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t key_cb_floats(int R) { return static_cast<size_t>(kGroups) * R * kCodes * kCodeword; }
+size_t val_cb_floats(int R) { return static_cast<size_t>(kGroups) * R * kCodes * kVDims; }
+
+cvq_status check_shape(const cvq_shape* s) {
+  if (s == nullptr) return CVQ_ERR_NULL;
+  if (s->head_dim != kHeadDim) return CVQ_ERR_UNSUPPORTED;
+  if (s->R != 1 && s->R != 2) return CVQ_ERR_UNSUPPORTED;
+  if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->t_cap < 0) return CVQ_ERR_SHAPE;
+  if (s->n_q_heads % s->n_kv_heads != 0) return CVQ_ERR_SHAPE;
+  if (s->batch > 65535 || s->n_q_heads > 65535) return CVQ_ERR_SHAPE;
+  if (!std::isfinite(s->rope_base) || !(s->rope_base > 1.0f)) return CVQ_ERR_SHAPE;
+  const int g = s->n_q_heads / s->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return CVQ_ERR_UNSUPPORTED;
+  return CVQ_OK;
+}
+
+cvq_status check_stride(int64_t stride, size_t per_head) {
+  if (stride < 0) return CVQ_ERR_SHAPE;
+  if (stride != 0 && static_cast<uint64_t>(stride) < per_head) return CVQ_ERR_SHAPE;
+  return CVQ_OK;
+}
+
+cvq_status check_ptr(const void* p) {
+  if (p == nullptr) return CVQ_ERR_NULL;
+  if (!aligned16(p)) return CVQ_ERR_ALIGN;
+  return CVQ_OK;
+}
+
+#define CVQ_TRY(expr)                 \
+  do {                                \
+    const cvq_status st_ = (expr);    \
+    if (st_ != CVQ_OK) return st_;    \
+  } while (0)
+
+cvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CVQ_OK : CVQ_ERR_CUDA; }
+
+cvq_status check_decode_common(const cvq_shape* s, const uint8_t* key_codes, const uint8_t* val_codes,
+                               const int32_t* seq_lens, const float* val_cb, int64_t val_stride,
+                               int n_splits, float* part_o, float* part_m, float* part_l) {
+  CVQ_TRY(check_ptr(key_codes));
+  CVQ_TRY(check_ptr(val_codes));
+  if (seq_lens == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0) return CVQ_ERR_ALIGN;
+  CVQ_TRY(check_ptr(val_cb));
+  CVQ_TRY(check_stride(val_stride, val_cb_floats(s->R)));
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  CVQ_TRY(check_ptr(part_o));
+  if (part_m == nullptr || part_l == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(part_m) & 3u) || (reinterpret_cast<uintptr_t>(part_l) & 3u))
+    return CVQ_ERR_ALIGN;
+  return CVQ_OK;
+}
+
+void fill_common(DecodeArgs& a, const cvq_shape* s, const uint8_t* key_codes, const uint8_t* val_codes,
+                 const int32_t* seq_lens, const float* val_cb, int64_t val_stride, int n_splits,
+                 float* part_o, float* part_m, float* part_l) {
+  a.key_codes = key_codes;
+  a.val_codes = val_codes;
+  a.seq_lens = seq_lens;
+  a.val_cb = val_cb;
+  a.val_cb_stride = val_stride;
+  a.batch = s->batch;
+  a.n_q_heads = s->n_q_heads;
+  a.n_kv_heads = s->n_kv_heads;
+  a.t_cap = s->t_cap;
+  a.n_splits = n_splits;
+  a.split_tokens = split_tokens_host(s->t_cap, n_splits);
+  a.part_o = part_o;
+  a.part_m = part_m;
+  a.part_l = part_l;
+  phase_turns_host(s->rope_base, &a.phase);
+}
+
+}  // namespace
+
+namespace cvq {
+
+void phase_turns_host(float rope_base, PhaseTurns* out) {
+  const long double two_pi = 6.283185307179586476925286766559L;
+  const long double base = static_cast<long double>(rope_base);
+  for (int j = 0; j < kPairs; ++j) {
+    const long double theta = powl(base, -2.0L * j / kHeadDim);
+    long double turns = theta / two_pi;                  // < 1 turn per token
+    turns -= floorl(turns);
+    const long double scaled = ldexpl(turns, 64);        // in [0, 2^64)
+    unsigned long long f;
+    if (scaled >= 18446744073709551615.0L) {
+      f = ~0ULL;
+    } else {
+      f = static_cast<unsigned long long>(scaled + 0.5L);
+    }
+    out->F[j] = f;
+  }
+}
+
+}  // namespace cvq
+
+extern "C" {
+
+const char* cvq_status_str(int status) {
+  switch (status) {
+    case CVQ_OK: return "CVQ_OK";
+    case CVQ_ERR_NULL: return "CVQ_ERR_NULL: a required pointer is NULL";
+    case CVQ_ERR_SHAPE: return "CVQ_ERR_SHAPE: inconsistent or out-of-range sizes";
+    case CVQ_ERR_ALIGN: return "CVQ_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case CVQ_ERR_UNSUPPORTED: return "CVQ_ERR_UNSUPPORTED: head_dim, R, dtype or GQA group not supported";
+    case CVQ_ERR_WORKSPACE: return "CVQ_ERR_WORKSPACE: n_splits out of range";
+    case CVQ_ERR_CUDA: return "CVQ_ERR_CUDA: the CUDA runtime reported an error";
+    default: return "unknown cvq_status";
+  }
+}
+
+int cvq_abi_version(void) { return CVQ_ABI_VERSION; }
+
+size_t cvq_ptable_bytes(const cvq_shape* s) {
+  if (check_shape(s) != CVQ_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->n_q_heads * key_cb_floats(s->R) * sizeof(float);
+}
+
+size_t cvq_partials_bytes(const cvq_shape* s, int n_splits) {
+  if (check_shape(s) != CVQ_OK || n_splits < 1 || n_splits > 4096) return 0;
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
+  return rows * (kHeadDim + 2) * sizeof(float);
+}
+
+int32_t cvq_split_tokens(const cvq_shape* s, int n_splits) {
+  if (check_shape(s) != CVQ_OK || n_splits < 1 || n_splits > 4096) return 0;
+  return split_tokens_host(s->t_cap, n_splits);
+}
+
+int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
+  if (check_shape(s) != CVQ_OK || sm_count < 1) return 1;
+  // aim for ~2 waves of CTAs over the SMs, each split at least 512 tokens long
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads;
+  long long want = (2LL * sm_count + units - 1) / units;
+  const long long max_by_len = (s->t_cap + 511) / 512;
+  if (want > max_by_len) want = max_by_len;
+  if (want < 1) want = 1;
+  if (want > 4096) want = 4096;
+  return static_cast<int>(want);
+}
+
+cvq_status cvq_qtable(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                      int64_t key_cb_head_stride, float* ptable, void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_ptr(q));
+  CVQ_TRY(check_ptr(key_cb));
+  CVQ_TRY(check_ptr(ptable));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
+  return from_cuda(launch_qtable(*s, q, q_dtype, key_cb, key_cb_head_stride, ptable,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+cvq_status cvq_decode_attn(const cvq_shape* s, const float* ptable, const uint8_t* key_codes,
+                           const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                           int64_t val_cb_head_stride, int n_splits, float* part_o, float* part_m,
+                           float* part_l, void* stream) {
+  CVQ_TRY(check_shape(s));
+  CVQ_TRY(check_ptr(ptable));
+  CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
+                              n_splits, part_o, part_m, part_l));
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fill_common(a, s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride, n_splits, part_o,
+              part_m, part_l);
+  a.key_tab = ptable;
+  a.key_tab_stride = static_cast<long long>(key_cb_floats(s->R));
+  return from_cuda(launch_decode_table(*s, a, static_cast<cudaStream_t>(stream)));
+}
+
+cvq_status cvq_decode_attn_gqa(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                               int64_t key_cb_head_stride, const uint8_t* key_codes,
+                               const uint8_t* val_codes, const int32_t* seq_lens,
+                               const float* val_cb, int64_t val_cb_head_stride, int n_splits,
+                               float* part_o, float* part_m, float* part_l, void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_ptr(q));
+  CVQ_TRY(check_ptr(key_cb));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
+  if ((s->n_q_heads / s->n_kv_heads) * s->R > 8) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
+                              n_splits, part_o, part_m, part_l));
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fill_common(a, s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride, n_splits, part_o,
+              part_m, part_l);
+  a.key_tab = key_cb;
+  a.key_tab_stride = key_cb_head_stride;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
+}
+
+cvq_status cvq_combine(const cvq_shape* s, int n_splits, const float* part_o, const float* part_m,
+                       const float* part_l, float* out, float* lse, void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  CVQ_TRY(check_ptr(part_o));
+  CVQ_TRY(check_ptr(out));
+  if (part_m == nullptr || part_l == nullptr || lse == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(part_m) & 3u) || (reinterpret_cast<uintptr_t>(part_l) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return CVQ_ERR_ALIGN;
+  return from_cuda(launch_combine(*s, n_splits, part_o, part_m, part_l, out, lse,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

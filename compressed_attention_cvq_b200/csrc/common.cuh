@@ -1,0 +1,99 @@
+// Shared definitions of the libcvq kernels: layout constants, the RoPE phase in exact
+// fixed-point turns, and small device helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cvq.h"
+
+namespace cvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kPairs = 64;
+constexpr int kGroups = 16;
+constexpr int kPairsPerGroup = 4;
+constexpr int kVDims = 8;
+constexpr int kCodes = 256;
+constexpr int kCodeword = 8;              // floats per key codeword (4 pairs x re/im)
+constexpr int kSplitAlign = 64;           // split boundaries are multiples of this
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// RoPE phase of pair j at position t as an exact fraction of a turn:
+//   theta_j t / (2 pi) mod 1  ==  (F_j * t mod 2^64) / 2^64,
+// with F_j = round(2^64 theta_j / (2 pi)).  The 64-bit wrap-around product performs
+// the range reduction exactly, so the angle stays accurate at any position
+// (theta_0 t reaches 1.3e5 rad at t = 131072, where an fp32 angle would be off by
+// up to ~8e-3 rad).
+struct PhaseTurns {
+  unsigned long long F[kPairs];
+};
+
+// Host: fill F_j for a RoPE base (long double for the 64-bit fraction).
+void phase_turns_host(float rope_base, PhaseTurns* out);
+
+// cos/sin of 2 pi * (turn64 / 2^64); the top 32 bits give the angle to 2^-32 turns,
+// taken as a signed value so the argument of the sine stays in [-pi, pi).
+__device__ __forceinline__ float2 phase_from_turn(unsigned long long turn64) {
+  const int hi = static_cast<int>(turn64 >> 32);
+  const float ang = static_cast<float>(hi) * 1.4629180792671596e-09f;  // 2 pi / 2^32
+  float s, c;
+  __sincosf(ang, &s, &c);
+  return make_float2(c, s);
+}
+
+__device__ __forceinline__ float2 phase_at(unsigned long long F, int t) {
+  return phase_from_turn(F * static_cast<unsigned long long>(static_cast<unsigned>(t)));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float load_q(const void* q, int q_dtype, size_t idx) {
+  if (q_dtype == CVQ_BF16) return bf16_bits_to_float(static_cast<const uint16_t*>(q)[idx]);
+  return static_cast<const float*>(q)[idx];
+}
+
+__device__ __forceinline__ int code_byte(const uint4& v, int G) {
+  const uint32_t w = (G < 4) ? v.x : (G < 8) ? v.y : (G < 12) ? v.z : v.w;
+  return static_cast<int>((w >> (8 * (G & 3))) & 0xffu);
+}
+
+// First token of split s and the split length (multiple of kSplitAlign).
+inline int32_t split_tokens_host(int32_t t_cap, int n_splits) {
+  int64_t c = (static_cast<int64_t>(t_cap) + n_splits - 1) / n_splits;
+  c = ((c + kSplitAlign - 1) / kSplitAlign) * kSplitAlign;
+  if (c < kSplitAlign) c = kSplitAlign;
+  return static_cast<int32_t>(c);
+}
+
+// Arguments shared by the decode kernels.
+struct DecodeArgs {
+  const float* key_tab;          // key codebook (per KV head) or P table (per query head)
+  long long key_tab_stride;      // floats between consecutive heads of key_tab
+  const void* q;                 // queries (GQA form only)
+  int q_dtype;
+  const uint8_t* key_codes;
+  const uint8_t* val_codes;
+  const int32_t* seq_lens;
+  const float* val_cb;
+  long long val_cb_stride;
+  int batch, n_q_heads, n_kv_heads, t_cap, n_splits, split_tokens;
+  float* part_o;
+  float* part_m;
+  float* part_l;
+  PhaseTurns phase;
+};
+
+// Launchers (defined next to their kernels).  Return cudaSuccess or the launch error.
+cudaError_t launch_qtable(const cvq_shape& s, const void* q, int q_dtype, const float* key_cb,
+                          long long key_cb_stride, float* ptable, cudaStream_t stream);
+cudaError_t launch_decode_table(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_gqa(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
+                           const float* part_m, const float* part_l, float* out, float* lse,
+                           cudaStream_t stream);
+
+}  // namespace cvq

@@ -1,0 +1,227 @@
+// Split-T flash-decode over the uint8 code stream: the straightforward form.
+//
+// One CTA = (split, head, sequence); one thread = one token of a 256-token tile.
+// Per token: gather the key codewords of every (group, round) from the table
+// (global memory, L1/L2 cached), sum the rounds, rotate by the RoPE phase
+// e^{i theta_j t} and project on the query head(s) -> score (in log2 units).
+// Online softmax per tile; the weights are accumulated per value code in
+// shared-memory bins (the CommVQ value reorder: softmax weights multiply the value
+// codes before the value codebook multiply -- review page, "forward_implications",
+// 4th item).  Epilogue: o = bins x val_cb.
+//
+// Table form (TABLE = true, NG = 1): key_tab is the P table of one query head and
+// the projection is the real part, Re(e^{i theta t} sum_r P).
+// GQA form (TABLE = false): key_tab is the key codebook of one KV head and the
+// projection is onto the NG query heads of its group, Re(conj(q) e^{i theta t} c).
+#include "common.cuh"
+
+namespace cvq {
+
+constexpr int kSimpleThreads = 256;
+
+template <int NG, int R, bool TABLE>
+__global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const DecodeArgs a) {
+  extern __shared__ float4 smem_f4[];
+  float* bins = reinterpret_cast<float*>(smem_f4);                // [NG][16][R][256]
+  __shared__ float qs[NG][kHeadDim];
+  __shared__ float red[kSimpleThreads / 32][NG];
+  __shared__ float tmax[NG];
+
+  const int split = blockIdx.x;
+  const int head = blockIdx.y;      // TABLE: query head; GQA: KV head
+  const int b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int group = a.n_q_heads / a.n_kv_heads;
+  const int h = TABLE ? head / group : head;     // KV head
+  const int hq0 = TABLE ? head : head * NG;       // first query head handled
+
+  int L = a.seq_lens[b];
+  L = L < 0 ? 0 : (L > a.t_cap ? a.t_cap : L);
+  const int t_begin = split * a.split_tokens;
+  const int t_end = min(t_begin + a.split_tokens, L);
+
+  const size_t part_row = (static_cast<size_t>(b) * a.n_q_heads + hq0) * a.n_splits + split;
+  if (t_begin >= t_end) {
+    for (int i = tid; i < NG * kHeadDim; i += kSimpleThreads) {
+      const int hh = i / kHeadDim;
+      a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + (i % kHeadDim)] = 0.f;
+    }
+    if (tid < NG) {
+      a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
+      a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
+    }
+    return;
+  }
+
+  const float qscale = kLog2e * 0.08838834764831845f;   // log2(e) / sqrt(128)
+  for (int i = tid; i < NG * kHeadDim; i += kSimpleThreads) {
+    const int hh = i / kHeadDim, d = i % kHeadDim;
+    float v;
+    if (TABLE) {
+      v = (d & 1) ? 0.f : qscale;
+    } else {
+      v = load_q(a.q, a.q_dtype, (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim + d) * qscale;
+    }
+    qs[hh][d] = v;
+  }
+  for (int i = tid; i < NG * kGroups * R * kCodes; i += kSimpleThreads) bins[i] = 0.f;
+
+  const float* tab = TABLE ? a.key_tab + (static_cast<size_t>(b) * a.n_q_heads + head) * a.key_tab_stride
+                           : a.key_tab + static_cast<size_t>(h) * a.key_tab_stride;
+  const size_t code_row = (static_cast<size_t>(b) * a.n_kv_heads + h) * a.t_cap;
+  const uint4* kcodes = reinterpret_cast<const uint4*>(a.key_codes) + code_row * R;
+  const uint4* vcodes = reinterpret_cast<const uint4*>(a.val_codes) + code_row * R;
+
+  float m_run[NG], l_run[NG];
+#pragma unroll
+  for (int hh = 0; hh < NG; ++hh) { m_run[hh] = -INFINITY; l_run[hh] = 0.f; }
+  __syncthreads();
+
+  for (int t0 = t_begin; t0 < t_end; t0 += kSimpleThreads) {
+    const int t = t0 + tid;
+    const bool valid = t < t_end;
+    uint4 kc[R], vc[R];
+    float s[NG];
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) s[hh] = -INFINITY;
+    if (valid) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        kc[r] = __ldg(kcodes + static_cast<size_t>(t) * R + r);
+        vc[r] = __ldg(vcodes + static_cast<size_t>(t) * R + r);
+      }
+#pragma unroll
+      for (int hh = 0; hh < NG; ++hh) s[hh] = 0.f;
+#pragma unroll 1
+      for (int G = 0; G < kGroups; ++G) {
+        float kr[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int c = code_byte(kc[r], G);
+          const float4* cw = reinterpret_cast<const float4*>(
+              tab + ((static_cast<size_t>(G) * R + r) * kCodes + c) * kCodeword);
+          const float4 lo = __ldg(cw), hi = __ldg(cw + 1);
+          kr[0] += lo.x; ki[0] += lo.y; kr[1] += lo.z; ki[1] += lo.w;
+          kr[2] += hi.x; ki[2] += hi.y; kr[3] += hi.z; ki[3] += hi.w;
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int j = 4 * G + p;
+          const float2 ph = phase_at(a.phase.F[j], t);
+          const float xr = ph.x * kr[p] - ph.y * ki[p];
+          const float xi = ph.y * kr[p] + ph.x * ki[p];
+#pragma unroll
+          for (int hh = 0; hh < NG; ++hh) s[hh] += qs[hh][2 * j] * xr + qs[hh][2 * j + 1] * xi;
+        }
+      }
+    }
+    // tile max per head
+    const int warp = tid / 32, lane = tid % 32;
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+      float v = s[hh];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+      if (lane == 0) red[warp][hh] = v;
+    }
+    __syncthreads();
+    if (tid < NG) {
+      float v = red[0][tid];
+      for (int w = 1; w < kSimpleThreads / 32; ++w) v = fmaxf(v, red[w][tid]);
+      tmax[tid] = v;
+    }
+    __syncthreads();
+    bool rescaled = false;
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+      const float m_new = fmaxf(m_run[hh], tmax[hh]);
+      if (m_new > m_run[hh]) {
+        const float sc = exp2f(m_run[hh] - m_new);
+        l_run[hh] *= sc;
+        float* bh = bins + hh * kGroups * R * kCodes;
+        for (int i = tid; i < kGroups * R * kCodes; i += kSimpleThreads) bh[i] *= sc;
+        m_run[hh] = m_new;
+        rescaled = true;
+      }
+    }
+    if (rescaled) __syncthreads();     // uniform: every thread sees the same tmax
+    if (valid) {
+#pragma unroll
+      for (int hh = 0; hh < NG; ++hh) {
+        const float w = exp2f(s[hh] - m_run[hh]);
+        l_run[hh] += w;
+        float* bh = bins + hh * kGroups * R * kCodes;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+          for (int G = 0; G < kGroups; ++G) {
+            atomicAdd(bh + (G * R + r) * kCodes + code_byte(vc[r], G), w);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // l: block sum per head
+  {
+    const int warp = tid / 32, lane = tid % 32;
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+      float v = l_run[hh];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) red[warp][hh] = v;
+    }
+    __syncthreads();
+    if (tid < NG) {
+      float v = 0.f;
+      for (int w = 0; w < kSimpleThreads / 32; ++w) v += red[w][tid];
+      a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = v;
+      a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = m_run[tid] * kLn2;
+    }
+  }
+  // epilogue: o[hh][8G + d] = sum_{r, c} bins[hh][G][r][c] * val_cb[G][r][c][d]
+  const float* vcb = a.val_cb + static_cast<size_t>(h) * a.val_cb_stride;
+  for (int i = tid; i < NG * kHeadDim; i += kSimpleThreads) {
+    const int hh = i / kHeadDim, dim = i % kHeadDim;
+    const int G = dim / kVDims, d = dim % kVDims;
+    const float* bh = bins + (hh * kGroups + G) * R * kCodes;
+    float acc = 0.f;
+    for (int rc = 0; rc < R * kCodes; ++rc) {
+      acc = fmaf(bh[rc], __ldg(vcb + (static_cast<size_t>(G) * R * kCodes + rc) * kVDims + d), acc);
+    }
+    a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + dim] = acc;
+  }
+}
+
+template <int NG, int R, bool TABLE>
+static cudaError_t launch_simple(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(NG) * kGroups * R * kCodes * sizeof(float);
+  auto k = decode_simple_kernel<NG, R, TABLE>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_splits, TABLE ? s.n_q_heads : s.n_kv_heads, s.batch);
+  k<<<grid, kSimpleThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_table(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  return s.R == 1 ? launch_simple<1, 1, true>(s, a, stream) : launch_simple<1, 2, true>(s, a, stream);
+}
+
+cudaError_t launch_decode_gqa(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  const int g = s.n_q_heads / s.n_kv_heads;
+  switch (g * 10 + s.R) {
+    case 11: return launch_simple<1, 1, false>(s, a, stream);
+    case 12: return launch_simple<1, 2, false>(s, a, stream);
+    case 21: return launch_simple<2, 1, false>(s, a, stream);
+    case 22: return launch_simple<2, 2, false>(s, a, stream);
+    case 41: return launch_simple<4, 1, false>(s, a, stream);
+    case 42: return launch_simple<4, 2, false>(s, a, stream);
+    case 81: return launch_simple<8, 1, false>(s, a, stream);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
+}  // namespace cvq

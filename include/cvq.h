@@ -1,0 +1,168 @@
+/*
+ * cvq.h -- C ABI of libcvq: CommVQ decode attention read directly from an additively
+ * vector-quantized KV cache whose key codebook commutes with RoPE.
+ *
+ * The method (CommVQ review page, pith.science arXiv 2506.18879, "key_machinery";
+ * CommVQ summary page, atlas.scime.ai, "Approach"): keys and values of the cache are
+ * stored as uint8 code indices into small additive codebooks.  A key codeword is a
+ * complex number c = a + ib per RoPE pair, i.e. the 2x2 block [[a,-b],[b,a]], which
+ * commutes with every RoPE rotation, so the query side can be combined with the
+ * codebook once per query and reused at every cached position.  Softmax weights are
+ * accumulated per value code before the value codebook multiply (review page,
+ * "forward_implications", 4th item).
+ *
+ * The instance implemented here:
+ *   head_dim 128 = 64 interleaved RoPE pairs (2j, 2j+1), theta_j = base^(-2j/128);
+ *   key:   16 groups of 4 pairs, R rounds, 256 complex codewords per (group, round);
+ *   value: 16 groups of 8 dims,  R rounds, 256 codewords per (group, round);
+ *   score_t = sum_j Re(e^{i theta_j t} conj(q_j) sum_r c_{t,r,j}) / sqrt(128), t = 0..L-1
+ *   out = sum_t softmax(score)_t v_t,   lse = ln sum_t exp(score_t).
+ * Query head hq reads KV head hq / (n_q_heads / n_kv_heads).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, row-major, and
+ *     16-byte aligned.  The library allocates nothing and keeps no state between calls.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream).  A status of CVQ_OK means the launch was accepted.
+ *   - Argument errors are detected on the host before any launch and returned as a
+ *     status; nothing is launched then.  Launch failures map to CVQ_ERR_CUDA.  No call
+ *     throws across the ABI.
+ *   - seq_lens[b] is read on the device and clamped to [0, t_cap].
+ */
+#ifndef CVQ_H
+#define CVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CVQ_API __attribute__((visibility("default")))
+#else
+#define CVQ_API
+#endif
+
+#define CVQ_ABI_VERSION 1
+#define CVQ_HEAD_DIM 128
+#define CVQ_GROUPS 16
+#define CVQ_CODES 256
+
+typedef enum {
+  CVQ_OK = 0,
+  CVQ_ERR_NULL = 1,        /* a required pointer is NULL                            */
+  CVQ_ERR_SHAPE = 2,       /* inconsistent or out-of-range sizes                    */
+  CVQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                      */
+  CVQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (head_dim != 128, R > 2 ...) */
+  CVQ_ERR_WORKSPACE = 5,   /* n_splits out of range                                 */
+  CVQ_ERR_CUDA = 6         /* the CUDA runtime reported an error                    */
+} cvq_status;
+
+typedef enum { CVQ_F32 = 0, CVQ_BF16 = 1 } cvq_dtype;
+
+typedef struct {
+  int32_t batch;      /* B  >= 1                                              */
+  int32_t n_q_heads;  /* Hq >= 1, a multiple of n_kv_heads                   */
+  int32_t n_kv_heads; /* Hkv >= 1; Hq/Hkv in {1, 2, 4, 8}                     */
+  int32_t head_dim;   /* must be 128                                          */
+  int32_t R;          /* residual rounds, 1 or 2                              */
+  int32_t t_cap;      /* token capacity of the code buffers per sequence, >= 0 */
+  float rope_base;    /* RoPE base, > 1 (500000 for LLaMA-3.1)                */
+} cvq_shape;
+
+/* Human-readable name of a status code (static storage). */
+CVQ_API const char* cvq_status_str(int status);
+
+/* CVQ_ABI_VERSION of the loaded library. */
+CVQ_API int cvq_abi_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_qtable -- the query x key-codebook table, built once per query.
+ *   (review page "key_machinery": query-dependent and codebook-dependent factors are
+ *    computed once and reused across all cached positions)
+ *
+ *   P[b, hq, G, r, c, p, 0:2] = conj(q_j) * c,  j = 4G + p,
+ *   q_j = q[b, hq, 2j] + i q[b, hq, 2j+1],  c = key_cb[h][G, r, c, p, 0] + i ...[1],
+ *   h = hq / (Hq / Hkv).  Unscaled (no 1/sqrt(128)).
+ *
+ *   q        [B, Hq, 128]           fp32 or bf16 (q_dtype), the already-rotated query
+ *   key_cb   [Hkv][16, R, 256, 4, 2] fp32; KV head h starts at key_cb + h * key_cb_head_stride
+ *            (stride in floats; 0 = one codebook shared by all KV heads, otherwise
+ *            >= 16*R*256*8)
+ *   ptable   [B, Hq, 16, R, 256, 4, 2] fp32 output, cvq_ptable_bytes(shape) bytes
+ * ------------------------------------------------------------------------------- */
+CVQ_API size_t cvq_ptable_bytes(const cvq_shape* shape);
+CVQ_API cvq_status cvq_qtable(const cvq_shape* shape, const void* q, int q_dtype, const float* key_cb,
+                      int64_t key_cb_head_stride, float* ptable, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Split-T partial states.  Split s of sequence b covers tokens
+ *   [s*C, min((s+1)*C, seq_len[b])),  C = cvq_split_tokens(shape, n_splits)
+ * (C is ceil(t_cap / n_splits) rounded up to a multiple of 64), so a split may be
+ * empty; an empty split stores m = -inf, l = 0, o = 0.
+ *   part_o [B, Hq, n_splits, 128]  sum_t e^{s_t - m} v_t   (unnormalized)
+ *   part_m [B, Hq, n_splits]       m = max_t s_t           (natural-log units)
+ *   part_l [B, Hq, n_splits]       l = sum_t e^{s_t - m}
+ * cvq_partials_bytes() is the total of the three arrays; 1 <= n_splits <= 4096.
+ * ------------------------------------------------------------------------------- */
+CVQ_API size_t cvq_partials_bytes(const cvq_shape* shape, int n_splits);
+CVQ_API int32_t cvq_split_tokens(const cvq_shape* shape, int n_splits);
+/* A split count that fills `sm_count` SMs for this shape (a suggestion). */
+CVQ_API int cvq_suggest_splits(const cvq_shape* shape, int sm_count);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_decode_attn -- split-T flash-decode over the code stream, table form.
+ *   (CommVQ summary page "Approach"; review page "key_machinery" and
+ *    "forward_implications" 4th item)
+ *   For each (b, hq, split): gather sum_r P[G, r, key_code, p] per pair, multiply by
+ *   the RoPE phase e^{i theta_j t}, take the real part and sum over pairs -> score;
+ *   online softmax; accumulate the weights per value code (bins[G, r, c]); finally
+ *   o = bins x val_cb.
+ *
+ *   ptable     output of cvq_qtable for the same shape
+ *   key_codes  [B, Hkv, t_cap, R, 16] uint8  (16-byte aligned)
+ *   val_codes  [B, Hkv, t_cap, R, 16] uint8
+ *   seq_lens   [B] int32 (device)
+ *   val_cb     [Hkv][16, R, 256, 8] fp32, KV head h at val_cb + h * val_cb_head_stride
+ *              (0 = shared, otherwise >= 16*R*256*8)
+ *   part_*     split partial states, see above
+ * ------------------------------------------------------------------------------- */
+CVQ_API cvq_status cvq_decode_attn(const cvq_shape* shape, const float* ptable, const uint8_t* key_codes,
+                           const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                           int64_t val_cb_head_stride, int n_splits, float* part_o, float* part_m,
+                           float* part_l, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_decode_attn_gqa -- the same partial states, computed per KV head for all of its
+ * Hq/Hkv query heads at once: each token's key codewords are gathered and rotated by
+ * the RoPE phase once (the codebook commutes with the rotation, so rotating the
+ * codeword equals rotating the key) and projected on every query head of the group.
+ *   Same score as cvq_decode_attn up to rounding:
+ *     Re(e^{i theta t} conj(q) c) = Re(conj(q) (e^{i theta t} c)).
+ *   q, q_dtype, key_cb, key_cb_head_stride as in cvq_qtable; the rest as in
+ *   cvq_decode_attn.
+ * ------------------------------------------------------------------------------- */
+CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, int q_dtype,
+                               const float* key_cb, int64_t key_cb_head_stride,
+                               const uint8_t* key_codes, const uint8_t* val_codes,
+                               const int32_t* seq_lens, const float* val_cb,
+                               int64_t val_cb_head_stride, int n_splits, float* part_o,
+                               float* part_m, float* part_l, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_combine -- merge split partial states (log-sum-exp):
+ *   M = max_s m_s;  L = sum_s l_s e^{m_s - M};
+ *   out[b, hq, :] = sum_s o_s e^{m_s - M} / L;   lse[b, hq] = M + ln L.
+ *   All splits empty (seq_len 0): out = 0, lse = -inf.
+ *   out [B, Hq, 128] fp32, lse [B, Hq] fp32.
+ * ------------------------------------------------------------------------------- */
+CVQ_API cvq_status cvq_combine(const cvq_shape* shape, int n_splits, const float* part_o,
+                       const float* part_m, const float* part_l, float* out, float* lse,
+                       void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CVQ_H */

@@ -1,0 +1,162 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+entry point include/cvq.h declares, reports sizes, and rejects bad arguments with a
+status before launching anything.  Every call below carries at least one invalid
+argument, so none of them reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_attention_cvq_b200 import _binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cvq.h")
+
+FAKE = 0x10000          # an aligned, non-null address that is never dereferenced
+MISALIGNED = 0x10008
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"CVQ_API\s+[\w\s\*]*?\b(cvq_\w+)\s*\(", src)))
+
+
+def _shape(**kw):
+    d = dict(batch=1, n_q_heads=32, n_kv_heads=8, R=2, t_cap=1024, rope_base=500000.0)
+    d.update(kw)
+    head_dim = d.pop("head_dim", 128)
+    return b.make_shape(d["batch"], d["n_q_heads"], d["n_kv_heads"], d["R"], d["t_cap"],
+                        d["rope_base"], head_dim)
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(b.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(b.EXPORTED)
+
+
+def test_abi_version_matches_header():
+    v = int(re.search(r"#define CVQ_ABI_VERSION (\d+)", open(HEADER).read()).group(1))
+    assert b.lib.cvq_abi_version() == v
+
+
+def test_status_strings():
+    for st, name in b.STATUS_NAMES.items():
+        assert b.status_str(st).startswith(name)
+    assert "unknown" in b.status_str(99)
+
+
+def test_sizes():
+    s = _shape()
+    assert b.lib.cvq_ptable_bytes(ctypes.byref(s)) == 1 * 32 * 16 * 2 * 256 * 8 * 4
+    assert b.lib.cvq_partials_bytes(ctypes.byref(s), 5) == 1 * 32 * 5 * 130 * 4
+    assert b.lib.cvq_partials_bytes(ctypes.byref(s), 0) == 0
+    assert b.lib.cvq_ptable_bytes(ctypes.byref(_shape(head_dim=64))) == 0
+
+
+@pytest.mark.parametrize("t_cap,n,expect", [(1024, 1, 1024), (1024, 3, 384), (4096, 16, 256),
+                                            (131072, 74, 1792), (1, 1, 64), (0, 4, 64),
+                                            (100, 7, 64)])
+def test_split_tokens(t_cap, n, expect):
+    c = b.lib.cvq_split_tokens(ctypes.byref(_shape(t_cap=t_cap)), n)
+    assert c == expect
+    assert c % 64 == 0 and c * n >= t_cap
+
+
+def test_suggest_splits_bounds():
+    for t in (0, 64, 4096, 131072):
+        n = b.lib.cvq_suggest_splits(ctypes.byref(_shape(t_cap=t)), 148)
+        assert 1 <= n <= 4096
+
+
+def _qtable(shape, q=FAKE, dt=0, kcb=FAKE, stride=0, P=FAKE):
+    return b.lib.cvq_qtable(ctypes.byref(shape) if shape is not None else None, q, dt, kcb,
+                            stride, P, None)
+
+
+def test_qtable_errors():
+    assert _qtable(None) == 1
+    assert _qtable(_shape(), q=None) == 1
+    assert _qtable(_shape(), P=MISALIGNED) == 3
+    assert _qtable(_shape(), dt=7) == 4
+    assert _qtable(_shape(head_dim=64)) == 4
+    assert _qtable(_shape(R=3)) == 4
+    assert _qtable(_shape(n_q_heads=12, n_kv_heads=8)) == 2
+    assert _qtable(_shape(n_q_heads=48, n_kv_heads=3)) == 4       # group of 16
+    assert _qtable(_shape(batch=0)) == 2
+    assert _qtable(_shape(t_cap=-1)) == 2
+    assert _qtable(_shape(rope_base=1.0)) == 2
+    assert _qtable(_shape(), stride=-5) == 2
+    assert _qtable(_shape(), stride=100) == 2                     # below one head's size
+
+
+def _decode(shape, n_splits=4, **kw):
+    a = dict(ptab=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, vcb=FAKE, vstride=0, po=FAKE, pm=FAKE, pl=FAKE)
+    a.update(kw)
+    return b.lib.cvq_decode_attn(ctypes.byref(shape), a["ptab"], a["kc"], a["vc"], a["lens"],
+                                 a["vcb"], a["vstride"], n_splits, a["po"], a["pm"], a["pl"], None)
+
+
+def test_decode_errors():
+    s = _shape()
+    assert _decode(s, ptab=None) == 1
+    assert _decode(s, kc=MISALIGNED) == 3
+    assert _decode(s, vc=None) == 1
+    assert _decode(s, lens=None) == 1
+    assert _decode(s, lens=FAKE + 2) == 3
+    assert _decode(s, n_splits=0) == 5
+    assert _decode(s, n_splits=5000) == 5
+    assert _decode(s, vstride=7) == 2
+    assert _decode(s, po=None) == 1
+    assert _decode(s, pm=FAKE + 1) == 3
+    assert _decode(_shape(head_dim=96)) == 4
+
+
+def _gqa(shape, n_splits=4, **kw):
+    a = dict(q=FAKE, dt=0, kcb=FAKE, kstride=0, kc=FAKE, vc=FAKE, lens=FAKE, vcb=FAKE, vstride=0,
+             po=FAKE, pm=FAKE, pl=FAKE)
+    a.update(kw)
+    return b.lib.cvq_decode_attn_gqa(ctypes.byref(shape), a["q"], a["dt"], a["kcb"], a["kstride"],
+                                     a["kc"], a["vc"], a["lens"], a["vcb"], a["vstride"], n_splits,
+                                     a["po"], a["pm"], a["pl"], None)
+
+
+def test_decode_gqa_errors():
+    s = _shape()
+    assert _gqa(s, q=None) == 1
+    assert _gqa(s, dt=2) == 4
+    assert _gqa(s, kcb=MISALIGNED) == 3
+    assert _gqa(s, kstride=1) == 2
+    assert _gqa(s, pl=None) == 1
+    assert _gqa(_shape(n_q_heads=64, n_kv_heads=8, R=2)) in (4,)    # group 8 with R = 2
+    assert _gqa(s, n_splits=-1) == 5
+
+
+def test_combine_errors():
+    s = _shape()
+    f = b.lib.cvq_combine
+    assert f(ctypes.byref(s), 0, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 5
+    assert f(ctypes.byref(s), 2, None, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(ctypes.byref(s), 2, FAKE, FAKE, FAKE, MISALIGNED, FAKE, None) == 3
+    assert f(ctypes.byref(s), 2, FAKE, FAKE, FAKE, FAKE, FAKE + 2, None) == 3
+    assert f(None, 2, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(b, "LIB_PATH", os.path.join(ROOT, "no_such_libcvq.so"))
+    with pytest.raises(ImportError):
+        b._load()
+
+
+def test_product_never_touches_oracle():
+    """Neither the package nor its C/CUDA sources refer to the oracle."""
+    pkg = os.path.join(ROOT, "compressed_attention_cvq_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"\boracle\b", src), fn
