@@ -16,7 +16,8 @@ CVQ_OK = 0
 CVQ_F32 = 0
 CVQ_BF16 = 1
 STATUS_NAMES = {0: "CVQ_OK", 1: "CVQ_ERR_NULL", 2: "CVQ_ERR_SHAPE", 3: "CVQ_ERR_ALIGN",
-                4: "CVQ_ERR_UNSUPPORTED", 5: "CVQ_ERR_WORKSPACE", 6: "CVQ_ERR_CUDA"}
+                4: "CVQ_ERR_UNSUPPORTED", 5: "CVQ_ERR_WORKSPACE", 6: "CVQ_ERR_CUDA",
+                7: "CVQ_ERR_STATIC_LIMIT"}
 
 
 class CvqError(RuntimeError):
@@ -49,6 +50,7 @@ def _load():
         "cvq_decode_attn": (I, [S, P, P, P, P, P, I64, I, P, P, P, P]),
         "cvq_decode_attn_gqa": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P, P]),
         "cvq_combine": (I, [S, I, P, P, P, P, P, P]),
+        "cvq_attend_static": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -71,7 +73,7 @@ class _LazyLib:
 lib = _LazyLib()
 EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partials_bytes",
             "cvq_split_tokens", "cvq_suggest_splits", "cvq_qtable", "cvq_decode_attn",
-            "cvq_decode_attn_gqa", "cvq_combine"]
+            "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static"]
 
 
 def status_str(st: int) -> str:

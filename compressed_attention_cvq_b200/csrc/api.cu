@@ -120,6 +120,7 @@ const char* cvq_status_str(int status) {
     case CVQ_ERR_UNSUPPORTED: return "CVQ_ERR_UNSUPPORTED: head_dim, R, dtype or GQA group not supported";
     case CVQ_ERR_WORKSPACE: return "CVQ_ERR_WORKSPACE: n_splits out of range";
     case CVQ_ERR_CUDA: return "CVQ_ERR_CUDA: the CUDA runtime reported an error";
+    case CVQ_ERR_STATIC_LIMIT: return "CVQ_ERR_STATIC_LIMIT: the partial states exceed the static scratch";
     default: return "unknown cvq_status";
   }
 }

@@ -1,0 +1,76 @@
+// cvq_attend_static: one decode step (GQA decode + combine) whose split partial states
+// live in a fixed, file-scope device array instead of caller-allocated memory.
+//
+// For callers that cannot allocate device memory while decoding: a serving process whose
+// memory pool has already claimed all free HBM for the KV cache, a plugin whose host
+// hands it no allocator, or a decode loop that cannot pay for cudaMalloc's implicit
+// synchronization.  They pass only inputs and outputs; the intermediate partial states
+// go to g_static_scratch, which every GPU that loads this library holds until exit.
+#include <mutex>
+
+#include "common.cuh"
+
+using namespace cvq;
+
+namespace {
+
+constexpr size_t kStaticScratchFloats = CVQ_STATIC_SCRATCH_BYTES / sizeof(float);
+static_assert(CVQ_STATIC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte alignment");
+
+// The partial states of the most recent call.  In host code this name is only a
+// stand-in for the symbol: its device address comes from cudaGetSymbolAddress.
+__device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
+
+constexpr int kMaxDevices = 128;
+float* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_static_scratch on the current device, looked up once per device
+// (with that device current) and cached.
+cudaError_t scratch_address(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" CVQ_API cvq_status cvq_attend_static(
+    const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+    int64_t key_cb_head_stride, const uint8_t* key_codes, const uint8_t* val_codes,
+    const int32_t* seq_lens, const float* val_cb, int64_t val_cb_head_stride, int n_splits,
+    float* out, float* lse, void* stream) {
+  if (out == nullptr || lse == nullptr) return CVQ_ERR_NULL;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return CVQ_ERR_ALIGN;
+  if (s == nullptr) return CVQ_ERR_NULL;
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  if (s->batch < 1 || s->n_q_heads < 1) return CVQ_ERR_SHAPE;
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
+  if (rows * (kHeadDim + 2) > kStaticScratchFloats) return CVQ_ERR_STATIC_LIMIT;
+
+  float* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return CVQ_ERR_CUDA;
+  // part_o [rows, 128], then part_m [rows], then part_l [rows]; every slot the combine
+  // reads is written by the decode of the same call, so nothing needs clearing.
+  float* part_o = base;
+  float* part_m = base + rows * kHeadDim;
+  float* part_l = part_m + rows;
+  const cvq_status st =
+      cvq_decode_attn_gqa(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
+                          seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
+                          stream);
+  if (st != CVQ_OK) return st;
+  return cvq_combine(s, n_splits, part_o, part_m, part_l, out, lse, stream);
+}

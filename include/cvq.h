@@ -57,7 +57,8 @@ typedef enum {
   CVQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                      */
   CVQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (head_dim != 128, R > 2 ...) */
   CVQ_ERR_WORKSPACE = 5,   /* n_splits out of range                                 */
-  CVQ_ERR_CUDA = 6         /* the CUDA runtime reported an error                    */
+  CVQ_ERR_CUDA = 6,        /* the CUDA runtime reported an error                    */
+  CVQ_ERR_STATIC_LIMIT = 7 /* cvq_attend_static: partials exceed the static scratch  */
 } cvq_status;
 
 typedef enum { CVQ_F32 = 0, CVQ_BF16 = 1 } cvq_dtype;
@@ -161,6 +162,32 @@ CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, in
 CVQ_API cvq_status cvq_combine(const cvq_shape* shape, int n_splits, const float* part_o,
                        const float* part_m, const float* part_l, float* out, float* lse,
                        void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_attend_static -- cvq_decode_attn_gqa followed by cvq_combine, with the split
+ * partial states kept in a fixed device array inside the library instead of memory
+ * the caller allocates.  The paper has no counterpart: this is an interface for
+ * callers that cannot allocate device memory while decoding -- a serving process
+ * whose pool has already claimed all free HBM for the KV cache, a plugin whose host
+ * gives it no allocator, or a decode loop that cannot afford cudaMalloc's implicit
+ * synchronization.  The call itself allocates nothing.
+ *
+ *   Arguments as in cvq_decode_attn_gqa, then out [B, Hq, 128] and lse [B, Hq] as in
+ *   cvq_combine.  B * Hq * n_splits * 130 * 4 bytes must fit in
+ *   CVQ_STATIC_SCRATCH_BYTES (4 MiB, held by every GPU that loads the library until
+ *   the process exits); larger calls return CVQ_ERR_STATIC_LIMIT before any launch.
+ *   The first call on a device looks up the array's device address with that device
+ *   current (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *   Every call reuses the same array: calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on it and must be serialized by the caller.
+ * ------------------------------------------------------------------------------- */
+#define CVQ_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+CVQ_API cvq_status cvq_attend_static(const cvq_shape* shape, const void* q, int q_dtype,
+                                     const float* key_cb, int64_t key_cb_head_stride,
+                                     const uint8_t* key_codes, const uint8_t* val_codes,
+                                     const int32_t* seq_lens, const float* val_cb,
+                                     int64_t val_cb_head_stride, int n_splits, float* out,
+                                     float* lse, void* stream);
 
 #ifdef __cplusplus
 }
