@@ -1,6 +1,7 @@
 // libcvq C ABI: argument validation on the host, then kernel launches.  Nothing is
 // allocated and no state is kept; every error is returned as a cvq_status before any
 // launch.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -145,14 +146,21 @@ int32_t cvq_split_tokens(const cvq_shape* s, int n_splits) {
 
 int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
   if (check_shape(s) != CVQ_OK || sm_count < 1) return 1;
-  // aim for ~2 waves of CTAs over the SMs, each split at least 512 tokens long
-  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads;
-  long long want = (2LL * sm_count + units - 1) / units;
-  const long long max_by_len = (s->t_cap + 511) / 512;
-  if (want > max_by_len) want = max_by_len;
-  if (want < 1) want = 1;
-  if (want > 4096) want = 4096;
-  return static_cast<int>(want);
+  // CTAs per split index and CTA slots on the GPU: the 4-head kernel runs a cluster of 2
+  // CTAs per (sequence, KV head, split), 2 per SM at R = 1 and 1 per SM at R = 2; the
+  // plain kernel runs one CTA per (sequence, KV head, split).  Take the fewest splits
+  // (longest, so the per-CTA codebook load and epilogue are amortized) whose CTAs fill
+  // at least 90% of their last wave.
+  const bool clustered = (s->n_q_heads / s->n_kv_heads) == 4;
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads * (clustered ? 2 : 1);
+  const long long slots = static_cast<long long>(sm_count) * (clustered && s->R == 1 ? 2 : 1);
+  const long long max_splits = std::max(1LL, std::min(4096LL, (s->t_cap + 255LL) / 256LL));
+  for (long long n = 1; n <= max_splits; ++n) {
+    const long long ctas = units * n;
+    const long long waves = (ctas + slots - 1) / slots;
+    if (ctas * 10 >= waves * slots * 9) return static_cast<int>(n);
+  }
+  return static_cast<int>(max_splits);
 }
 
 cvq_status cvq_qtable(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,

@@ -92,6 +92,8 @@ cudaError_t launch_qtable(const cvq_shape& s, const void* q, int q_dtype, const 
                           long long key_cb_stride, float* ptable, cudaStream_t stream);
 cudaError_t launch_decode_table(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_gqa(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+// the clustered kernel for 4 query heads per KV head (decode_gqa.cu)
+cudaError_t launch_decode_gqa4(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
                            const float* part_m, const float* part_l, float* out, float* lse,
                            cudaStream_t stream);

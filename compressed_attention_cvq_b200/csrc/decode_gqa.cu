@@ -1,0 +1,382 @@
+// Split-T flash-decode over the uint8 code stream, GQA form, for groups of 4 query
+// heads per KV head (the LLaMA-3.1-8B shape).
+//
+// Work unit: one (sequence b, KV head h, split s), handled by a cluster of two CTAs.
+// CTA rank g of the pair owns key/value groups 8g .. 8g+7, so its shared memory holds
+// half of each codebook (64R KiB of key codewords, 32R KiB of value bins) and both
+// residual depths fit on chip.
+//
+// Per token and KV head (CommVQ review page, "key_machinery" and "forward_implications"):
+//   1. gather sum_r c[G, r, key_code] for the CTA's 8 groups (8 lanes per token, one
+//      group = 4 RoPE pairs per lane);
+//   2. rotate by the RoPE phase e^{i theta_j t} -- the codeword commutes with the rotation,
+//      so this equals rotating the key -- and project on the 4 query heads;
+//   3. reduce the partial scores over the token's 8 lanes, exchange them with the peer
+//      CTA through distributed shared memory and add: the score of every head;
+//   4. online softmax with a reference max per head that is raised only when a tile's
+//      max exceeds it by more than 8 (log2 units), so the bins are rescaled rarely;
+//   5. add the weight of every head to the bin of the token's value code, per group and
+//      round (the value reorder: weights multiply value codes before the codebook);
+//   6. epilogue: o = bins x value codebook for the CTA's 64 output dims.
+//
+// Shared-memory layouts, chosen for conflict-free access (32 banks x 4 bytes):
+//   key / value codewords: 16-byte chunk ((r*256 + c)*2 + half)*8 + G_local, so the 8
+//     lanes of a quarter-warp (one token, groups 0..7) hit 8 different bank groups;
+//   bins: float ((r*256 + c)*4 + head)*8 + G_local; at every atomic step the 32 lanes
+//     of a warp (4 tokens x 4 heads x 2 group halves, each token on a rotated group)
+//     touch 32 different banks and never the same address.
+//
+// Tokens: kSlots = 4 per warp per step; slot sigma handles t_begin + sigma + kSlots*j.
+// The phase of a lane's 4 pairs starts from the exact fixed-point turn and advances by
+// e^{i theta_j kSlots} per step (rounding error ~1e-7 per step).  Code bytes of the
+// next tile are copied to shared memory with cp.async while the current tile computes.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace cvq {
+
+namespace {
+
+constexpr int kHeads = 4;              // query heads per KV head
+constexpr int kLocalGroups = 8;        // groups per CTA of the pair
+constexpr int kTile = 256;             // tokens per tile (softmax / exchange period)
+constexpr float kRescaleSlack = 8.0f;  // log2 units the reference max may lag behind
+
+template <int R>
+struct Cfg {
+  static constexpr int kThreads = (R == 1) ? 256 : 512;
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kSlots = kWarps * 4;                  // tokens per step
+  static constexpr int kSteps = kTile / kSlots;              // steps per tile
+  static constexpr int kMinBlocks = (R == 1) ? 2 : 1;
+  static constexpr int kCodeChunks = R * kCodes * 2 * kLocalGroups;   // 16-byte chunks
+  static constexpr int kBins = R * kCodes * kHeads * kLocalGroups;    // floats
+  static constexpr int kXchg = 2 * kTile * kHeads;                    // floats (2 buffers)
+  static constexpr int kCodeBytes = 2 * kTile * R * 16;               // 2 buffers x (key 8 B + val 8 B) x R
+  static constexpr size_t kSmem = sizeof(float4) * kCodeChunks +
+                                  sizeof(float) * (kBins + kXchg + kWarps * kHeads + 2 * kHeads) +
+                                  kCodeBytes;
+  static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+
+template <int R>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cfg<R>::kMinBlocks)
+    decode_gqa4_kernel(const DecodeArgs a) {
+  using C = Cfg<R>;
+  extern __shared__ float4 smem4[];
+  float4* cw_s = smem4;                                               // [R][256][2][8] chunks
+  float* bins = reinterpret_cast<float*>(smem4 + C::kCodeChunks);     // [R][256][4][8]
+  float* xchg = bins + C::kBins;                                      // [2][kTile][4]
+  float* red = xchg + C::kXchg;                                       // [kWarps][4]
+  float* fh = red + C::kWarps * kHeads;                               // [4] tile max / factors
+  float* mtile = fh + kHeads;                                         // [4]
+  uint8_t* code_s = reinterpret_cast<uint8_t*>(mtile + kHeads);       // [2][kTile][R][key 8 | val 8]
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());           // which half of the groups
+  const int split = blockIdx.x >> 1;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int tau = lane >> 3;               // token slot within the warp (0..3)
+  const int k = lane & 7;                  // local group of the key side
+  const int hk = k & 3;                    // head whose score / weights this lane keeps
+  const int gh = k >> 2;                   // which 4 local groups this lane bins
+  const int sigma = warp * 4 + tau;        // token slot within the step
+  const int hq0 = h * kHeads;
+
+  int L = a.seq_lens[b];
+  L = L < 0 ? 0 : (L > a.t_cap ? a.t_cap : L);
+  const int t_begin = split * a.split_tokens;
+  const int t_end = min(t_begin + a.split_tokens, L);
+  const size_t part_row = (static_cast<size_t>(b) * a.n_q_heads + hq0) * a.n_splits + split;
+
+  if (t_begin >= t_end) {   // both CTAs of the pair take this branch together
+    for (int i = tid; i < kHeads * 64; i += C::kThreads) {
+      const int hh = i >> 6, d = i & 63;
+      a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + rank * 64 + d] = 0.f;
+    }
+    if (rank == 0 && tid < kHeads) {
+      a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
+      a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
+    }
+    return;
+  }
+
+  const size_t code_row = (static_cast<size_t>(b) * a.n_kv_heads + h) * a.t_cap;
+  // copy the code bytes of this CTA's 8 groups for one tile (key and value, every round)
+  auto stage_codes = [&](int t_tile, int buf) {
+    for (int i = tid; i < kTile * R; i += C::kThreads) {
+      const int tt = i % kTile, r = i / kTile;
+      const int t = t_tile + tt;
+      if (t < t_end) {
+        const size_t off = (code_row + t) * (16 * R) + r * 16 + rank * 8;
+        uint8_t* dst = code_s + ((buf * kTile + tt) * R + r) * 16;
+        cp_async8(dst, a.key_codes + off);
+        cp_async8(dst + 8, a.val_codes + off);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // ---- prologue: key codewords of this CTA's groups, first tile's codes (async) ----
+  const float4* kcb = reinterpret_cast<const float4*>(a.key_tab + static_cast<size_t>(h) * a.key_tab_stride);
+  for (int i = tid; i < C::kCodeChunks; i += C::kThreads) {
+    const int gl = i & 7, half = (i >> 3) & 1, c = (i >> 4) & 255, r = i >> 12;
+    const int G = rank * kLocalGroups + gl;
+    cp_async16(cw_s + i, kcb + ((static_cast<size_t>(G) * R + r) * kCodes + c) * 2 + half);
+  }
+  stage_codes(t_begin, 0);
+  for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] = 0.f;
+
+  // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2 units
+  const float qscale = kLog2e * 0.08838834764831845f;
+  const int G = rank * kLocalGroups + k;
+  float2 qv[kHeads][4];
+#pragma unroll
+  for (int hh = 0; hh < kHeads; ++hh) {
+    const size_t qb = (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim + 8 * G;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      qv[hh][p] = make_float2(load_q(a.q, a.q_dtype, qb + 2 * p) * qscale,
+                              load_q(a.q, a.q_dtype, qb + 2 * p + 1) * qscale);
+    }
+  }
+  float2 ph[4], adv[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    ph[p] = phase_at(a.phase.F[4 * G + p], t_begin + sigma);
+    adv[p] = phase_at(a.phase.F[4 * G + p], C::kSlots);
+  }
+  float* peer_xchg = cluster.map_shared_rank(xchg, rank ^ 1);
+
+  float m_ref = -INFINITY;      // reference max (log2 units) of head hk; equal in all lanes
+  float l_acc = 0.f;            // this lane's share of sum_t w for head hk
+
+  cp_async_wait_all();
+  cluster.sync();               // codewords, bins and the first codes ready in both CTAs
+
+  const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int t_tile = t_begin + tile * kTile;
+    const int buf = tile & 1;
+    if (tile > 0) {
+      cp_async_wait_all();      // this tile's codes (issued one tile ago) have landed
+      __syncthreads();          // ... for every thread; the other buffer is free again
+    }
+    if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
+    const uint8_t* cb = code_s + static_cast<size_t>(buf) * kTile * R * 16;
+    float* xb = xchg + buf * (kTile * kHeads);
+    float* pxb = peer_xchg + buf * (kTile * kHeads);
+
+    float s_part[C::kSteps];
+#pragma unroll
+    for (int st = 0; st < C::kSteps; ++st) {
+      const int tt = st * C::kSlots + sigma;             // token within the tile
+      float2 kw[4];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int c = cb[(tt * R + r) * 16 + k];
+        const float4* src = cw_s + ((r * kCodes + c) * 2) * kLocalGroups + k;
+        const float4 lo = src[0], hi = src[kLocalGroups];
+        if (r == 0) {
+          kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
+          kw[2] = make_float2(hi.x, hi.y); kw[3] = make_float2(hi.z, hi.w);
+        } else {
+          kw[0].x += lo.x; kw[0].y += lo.y; kw[1].x += lo.z; kw[1].y += lo.w;
+          kw[2].x += hi.x; kw[2].y += hi.y; kw[3].x += hi.z; kw[3].y += hi.w;
+        }
+      }
+      float2 part2[kHeads];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 x = cmul(ph[p], kw[p]);
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh)
+          part2[hh] = p == 0 ? __fmul2_rn(qv[hh][p], x) : __ffma2_rn(qv[hh][p], x, part2[hh]);
+        ph[p] = cmul(ph[p], adv[p]);
+      }
+      float part[kHeads];
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) part[hh] = part2[hh].x + part2[hh].y;
+      // sum the 4 head partials over the token's 8 lanes; lanes k, k^4 keep head k & 3
+      const bool b1 = (k & 2) != 0;
+      const float r0 = (b1 ? part[2] : part[0]) + __shfl_xor_sync(0xffffffffu, b1 ? part[0] : part[2], 2);
+      const float r1 = (b1 ? part[3] : part[1]) + __shfl_xor_sync(0xffffffffu, b1 ? part[1] : part[3], 2);
+      const bool b0 = (k & 1) != 0;
+      float v = (b0 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b0 ? r0 : r1, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      s_part[st] = v;
+      if (k < 4) pxb[tt * kHeads + hk] = v;
+    }
+    cluster.sync();   // the peer's partials of this tile have landed in xb
+
+    // full scores (the same order of addition in both CTAs -> identical values)
+    float s[C::kSteps];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int st = 0; st < C::kSteps; ++st) {
+      const int tt = st * C::kSlots + sigma;
+      const float other = xb[tt * kHeads + hk];
+      const float v = rank == 0 ? s_part[st] + other : other + s_part[st];
+      s[st] = (t_tile + tt < t_end) ? v : -INFINITY;
+      mx = fmaxf(mx, s[st]);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (lane < kHeads) red[warp * kHeads + lane] = mx;
+    __syncthreads();
+    if (tid < kHeads) {
+      float v = red[tid];
+#pragma unroll
+      for (int w = 1; w < C::kWarps; ++w) v = fmaxf(v, red[w * kHeads + tid]);
+      mtile[tid] = v;
+    }
+    __syncthreads();
+    bool any_rescale = false;
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh) {
+      const float m_old = __shfl_sync(0xffffffffu, m_ref, hh);   // lane hh keeps head hh
+      any_rescale |= (m_old == -INFINITY) || (mtile[hh] > m_old + kRescaleSlack);
+    }
+    if (any_rescale) {   // uniform: every thread read the same mtile
+      const float m_new = (m_ref == -INFINITY || mtile[hk] > m_ref + kRescaleSlack) ? mtile[hk] : m_ref;
+      const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
+      l_acc *= f;
+      m_ref = m_new;
+      if (tid < kHeads) fh[tid] = f;   // thread tid < 4 is lane tid: head tid
+      __syncthreads();
+      for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] *= fh[(i >> 3) & 3];
+      __syncthreads();
+    }
+    // weights: lanes with k < 4 exponentiate the first half of the steps, the others the
+    // second half; each lane then holds the weights of all steps of its token slot
+    float w[C::kSteps];
+#pragma unroll
+    for (int st = 0; st < C::kSteps; ++st) {
+      const bool mine = (st < C::kSteps / 2) == (gh == 0);
+      float e = 0.f;
+      if (mine) {
+        e = exp2f(s[st] - m_ref);     // 0 for tokens past the end (s = -inf)
+        l_acc += e;
+      }
+      w[st] = e + __shfl_xor_sync(0xffffffffu, e, 4);
+    }
+    // value-code bins: lane bins head hk for local groups 4 gh .. 4 gh + 3 (rotated by tau)
+#pragma unroll
+    for (int st = 0; st < C::kSteps; ++st) {
+      const int tt = st * C::kSlots + sigma;
+      if (t_tile + tt < t_end) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t word = *reinterpret_cast<const uint32_t*>(cb + (tt * R + r) * 16 + 8 + 4 * gh);
+          const uint32_t rot = __funnelshift_r(word, word, 8 * tau);   // byte i: group 4gh + ((i + tau) & 3)
+          float* bin_r = bins + r * (kCodes * kHeads * kLocalGroups) + hk * kLocalGroups + 4 * gh;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = (rot >> (8 * i)) & 0xff;
+            atomicAdd(bin_r + c * (kHeads * kLocalGroups) + ((i + tau) & 3), w[st]);
+          }
+        }
+      }
+    }
+  }
+
+  // ---- l: lanes hold disjoint shares of head hk; sum over slots, halves and warps ----
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 4);
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 8);
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 16);
+  __syncthreads();                                   // every bin update is done
+  if (lane < kHeads) red[warp * kHeads + lane] = l_acc;
+  __syncthreads();
+  if (rank == 0 && tid < kHeads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < C::kWarps; ++w) v += red[w * kHeads + tid];
+    a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = v;
+    a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = m_ref * kLn2;   // lane tid: head tid
+  }
+
+  // ---- epilogue: o[head][8 G + d] = sum_{r,c} bins[r][c][head][G] * val_cb[G][r][c][d] ----
+  // value codewords of this CTA's groups replace the key codewords, same chunk layout
+  const float4* vcb = reinterpret_cast<const float4*>(a.val_cb + static_cast<size_t>(h) * a.val_cb_stride);
+  for (int i = tid; i < C::kCodeChunks; i += C::kThreads) {
+    const int gl = i & 7, half = (i >> 3) & 1, c = (i >> 4) & 255, r = i >> 12;
+    const int Gv = rank * kLocalGroups + gl;
+    cp_async16(cw_s + i, vcb + ((static_cast<size_t>(Gv) * R + r) * kCodes + c) * 2 + half);
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  {
+    // warp = slice of codes, lane = (head, local group): bins reads are 32 consecutive
+    // floats, codeword reads 8 distinct chunks in 8 bank groups
+    const int gl = lane & 7, hh = lane >> 3;
+    constexpr int kPerSlice = R * kCodes / C::kWarps;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int ci = 0; ci < kPerSlice; ++ci) {
+      const int rc = warp * kPerSlice + ci;            // r * 256 + c
+      const float wgt = bins[(rc * kHeads + hh) * kLocalGroups + gl];
+      const float4 v0 = cw_s[(rc * 2) * kLocalGroups + gl];
+      const float4 v1 = cw_s[(rc * 2 + 1) * kLocalGroups + gl];
+      acc[0] = fmaf(wgt, v0.x, acc[0]); acc[1] = fmaf(wgt, v0.y, acc[1]);
+      acc[2] = fmaf(wgt, v0.z, acc[2]); acc[3] = fmaf(wgt, v0.w, acc[3]);
+      acc[4] = fmaf(wgt, v1.x, acc[4]); acc[5] = fmaf(wgt, v1.y, acc[5]);
+      acc[6] = fmaf(wgt, v1.z, acc[6]); acc[7] = fmaf(wgt, v1.w, acc[7]);
+    }
+    __syncthreads();                                   // bins no longer read: reuse them
+    float* part_s = bins;                              // [kWarps][32 lanes][8]
+#pragma unroll
+    for (int d = 0; d < 8; ++d) part_s[(warp * 32 + lane) * 8 + d] = acc[d];
+    __syncthreads();
+    for (int o = tid; o < kHeads * kLocalGroups * 8; o += C::kThreads) {
+      const int d = o & 7, ln = o >> 3;                // ln = head * 8 + local group
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < C::kWarps; ++w) v += part_s[(w * 32 + ln) * 8 + d];
+      const int hh2 = ln >> 3, gl2 = ln & 7;
+      a.part_o[(part_row + static_cast<size_t>(hh2) * a.n_splits) * kHeadDim +
+               8 * (rank * kLocalGroups + gl2) + d] = v;
+    }
+  }
+  cluster.sync();   // no CTA leaves while its peer may still address its shared memory
+}
+
+template <int R>
+cudaError_t launch_gqa4(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  const size_t smem = Cfg<R>::kSmem;
+  auto k = decode_gqa4_kernel<R>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(2 * a.n_splits, s.n_kv_heads, s.batch);
+  k<<<grid, Cfg<R>::kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_gqa4(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  return s.R == 1 ? launch_gqa4<1>(s, a, stream) : launch_gqa4<2>(s, a, stream);
+}
+
+}  // namespace cvq

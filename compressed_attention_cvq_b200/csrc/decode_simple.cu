@@ -217,8 +217,8 @@ cudaError_t launch_decode_gqa(const cvq_shape& s, const DecodeArgs& a, cudaStrea
     case 12: return launch_simple<1, 2, false>(s, a, stream);
     case 21: return launch_simple<2, 1, false>(s, a, stream);
     case 22: return launch_simple<2, 2, false>(s, a, stream);
-    case 41: return launch_simple<4, 1, false>(s, a, stream);
-    case 42: return launch_simple<4, 2, false>(s, a, stream);
+    case 41:
+    case 42: return launch_decode_gqa4(s, a, stream);
     case 81: return launch_simple<8, 1, false>(s, a, stream);
     default: return cudaErrorInvalidConfiguration;
   }

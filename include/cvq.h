@@ -104,8 +104,11 @@ CVQ_API cvq_status cvq_qtable(const cvq_shape* shape, const void* q, int q_dtype
  * (C is ceil(t_cap / n_splits) rounded up to a multiple of 64), so a split may be
  * empty; an empty split stores m = -inf, l = 0, o = 0.
  *   part_o [B, Hq, n_splits, 128]  sum_t e^{s_t - m} v_t   (unnormalized)
- *   part_m [B, Hq, n_splits]       m = max_t s_t           (natural-log units)
+ *   part_m [B, Hq, n_splits]       reference m, natural-log units, with
+ *                                  max_t s_t - 8 ln 2 <= m <= max_t s_t
  *   part_l [B, Hq, n_splits]       l = sum_t e^{s_t - m}
+ * (m may lag the split maximum by up to 8 ln 2 so that the decode rescales its
+ * accumulators rarely; m + ln l and o / l do not depend on it.)
  * cvq_partials_bytes() is the total of the three arrays; 1 <= n_splits <= 4096.
  * ------------------------------------------------------------------------------- */
 CVQ_API size_t cvq_partials_bytes(const cvq_shape* shape, int n_splits);

@@ -109,8 +109,8 @@ def test_seq_lens_clamped_to_capacity():
 
 @pytest.mark.parametrize("form", FORMS)
 def test_partials_follow_documented_split_rule(form):
-    """Each split's (m, l, o) equals the oracle's partial state over tokens
-    [s*C, min((s+1)*C, L)), C = cvq_split_tokens."""
+    """Each split's (m, l, o) is the oracle's partial state over tokens
+    [s*C, min((s+1)*C, L)), C = cvq_split_tokens, up to the choice of reference m."""
     d = _small(batch=1, n_q_heads=4, n_kv_heads=1, t_cap=1000, R=1, seed=21)
     dd = to_device(d)
     shape = cvq.shape_of(dd["q"], dd["key_codes"])
@@ -133,10 +133,12 @@ def test_partials_follow_documented_split_rule(form):
             if t1 <= t0:
                 assert np.isneginf(pm[0, hq, si]) and pl[0, hq, si] == 0
                 continue
-            assert abs(pm[0, hq, si] - m[si]) < 1e-4
-            # compare normalized states (m is a free reference point up to rounding)
-            f = math.exp(pm[0, hq, si] - m[si])
-            assert abs(pl[0, hq, si] - l[si] * f) / (l[si] * f) < 1e-4
+            # m is a reference point within [max - 8 ln 2, max]; the split's log-sum-exp
+            # m + ln l and its normalized output o / l do not depend on that choice
+            assert m[si] - 8 * math.log(2) - 1e-4 <= pm[0, hq, si] <= m[si] + 1e-4
+            lse_gpu = pm[0, hq, si] + math.log(pl[0, hq, si])
+            lse_ref = m[si] + math.log(l[si])
+            assert abs(lse_gpu - lse_ref) / max(1.0, abs(lse_ref)) < 1e-4
             np.testing.assert_allclose(po[0, hq, si] / pl[0, hq, si], o[si] / l[si], atol=2e-3)
 
 
