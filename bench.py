@@ -58,6 +58,25 @@ def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
     return codes + cbs
 
 
+def recorded_traffic(workload: str, form: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu record, if it was
+    taken on this workload and the kernel source has not changed since (else None)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if form != "gqa" or not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, rec["source"])
+    if rec.get("workload") != workload or not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -328,7 +347,8 @@ def run_gpu(args):
             "code_hbm_frac": bytes_ / (dec_mean_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
             "roofline": {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak_tflops,
                          "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
-                         "traffic": None,
+                         "traffic": recorded_traffic(args.workload, args.form),
+                         "traffic_unit": "DRAM bytes per decode launch (ncu)",
                          "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {sm_max:.0f} MHz "
                                         f"(unit counts and max clock; HBM peak {pk_src})"},
             "e2e": {"value": world * total_tokens / (e2e_ms * 1e-3), "unit": "KV tokens/s per layer",

@@ -32,6 +32,8 @@
 // next tile are copied to shared memory with cp.async while the current tile computes.
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -72,6 +74,13 @@ __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
   return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
@@ -148,17 +157,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   stage_codes(t_begin, 0);
   for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] = 0.f;
 
-  // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2 units
+  // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2
+  // units.  Slot j holds head (k ^ j) & 3: with this lane-dependent order the butterfly
+  // that sums the partials over the token's 8 lanes needs no selects, and leaves head
+  // k & 3 in lanes k and k ^ 4.
   const float qscale = kLog2e * 0.08838834764831845f;
   const int G = rank * kLocalGroups + k;
   float2 qv[kHeads][4];
 #pragma unroll
-  for (int hh = 0; hh < kHeads; ++hh) {
+  for (int j = 0; j < kHeads; ++j) {
+    const int hh = (k ^ j) & 3;
     const size_t qb = (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim + 8 * G;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      qv[hh][p] = make_float2(load_q(a.q, a.q_dtype, qb + 2 * p) * qscale,
-                              load_q(a.q, a.q_dtype, qb + 2 * p + 1) * qscale);
+      qv[j][p] = make_float2(load_q(a.q, a.q_dtype, qb + 2 * p) * qscale,
+                             load_q(a.q, a.q_dtype, qb + 2 * p + 1) * qscale);
     }
   }
   float2 ph[4], adv[4];
@@ -175,15 +188,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   cp_async_wait_all();
   cluster.sync();               // codewords, bins and the first codes ready in both CTAs
 
+  // per-lane float offsets into the bins: step i of a token's atomics adds to local group
+  // 4 gh + ((i + tau) & 3) of head hk
+  int bin_off[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) bin_off[i] = hk * kLocalGroups + 4 * gh + ((i + tau) & 3);
+
   const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
-  for (int tile = 0; tile < n_tiles; ++tile) {
-    const int t_tile = t_begin + tile * kTile;
-    const int buf = tile & 1;
-    if (tile > 0) {
-      cp_async_wait_all();      // this tile's codes (issued one tile ago) have landed
-      __syncthreads();          // ... for every thread; the other buffer is free again
+
+  // Software pipeline over tiles.  Iteration t: key side of tile t -> arrive on the
+  // cluster barrier -> bin atomics of tile t-1 (weights and value codes kept in
+  // registers) -> wait on the barrier -> scores, max and weights of tile t.  The
+  // atomics overlap the exchange with the peer CTA.
+  float w[C::kSteps];            // weights of the previous tile's tokens (head hk)
+  uint32_t vw[C::kSteps][R];     // value code bytes of those tokens (groups 4 gh .. 4 gh + 3)
+  bool prev_valid[C::kSteps];
+#pragma unroll
+  for (int st = 0; st < C::kSteps; ++st) prev_valid[st] = false;
+
+  auto bin_atomics = [&]() {
+#pragma unroll
+    for (int st = 0; st < C::kSteps; ++st) {
+      if (prev_valid[st]) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t rot = __funnelshift_r(vw[st][r], vw[st][r], 8 * tau);  // byte i: group 4gh + ((i + tau) & 3)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = static_cast<int>(__byte_perm(rot, 0u, 0x4440u + i));
+            atomicAdd(bins + r * (kCodes * kHeads * kLocalGroups) + c * (kHeads * kLocalGroups) + bin_off[i],
+                      w[st]);
+          }
+        }
+      }
     }
-    if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
+  };
+
+  // one tile: FULL = every token of the tile is inside the split (no per-token checks)
+  auto run_tile = [&](const int t_tile, const int buf, auto full_tag) {
+    constexpr bool FULL = decltype(full_tag)::value;
     const uint8_t* cb = code_s + static_cast<size_t>(buf) * kTile * R * 16;
     float* xb = xchg + buf * (kTile * kHeads);
     float* pxb = peer_xchg + buf * (kTile * kHeads);
@@ -196,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int c = cb[(tt * R + r) * 16 + k];
-        const float4* src = cw_s + ((r * kCodes + c) * 2) * kLocalGroups + k;
+        const float4* src = cw_s + (r * kCodes + c) * (2 * kLocalGroups) + k;
         const float4 lo = src[0], hi = src[kLocalGroups];
         if (r == 0) {
           kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
@@ -211,24 +254,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
       for (int p = 0; p < 4; ++p) {
         const float2 x = cmul(ph[p], kw[p]);
 #pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh)
-          part2[hh] = p == 0 ? __fmul2_rn(qv[hh][p], x) : __ffma2_rn(qv[hh][p], x, part2[hh]);
+        for (int j = 0; j < kHeads; ++j)
+          part2[j] = p == 0 ? __fmul2_rn(qv[j][p], x) : __ffma2_rn(qv[j][p], x, part2[j]);
         ph[p] = cmul(ph[p], adv[p]);
       }
-      float part[kHeads];
-#pragma unroll
-      for (int hh = 0; hh < kHeads; ++hh) part[hh] = part2[hh].x + part2[hh].y;
-      // sum the 4 head partials over the token's 8 lanes; lanes k, k^4 keep head k & 3
-      const bool b1 = (k & 2) != 0;
-      const float r0 = (b1 ? part[2] : part[0]) + __shfl_xor_sync(0xffffffffu, b1 ? part[0] : part[2], 2);
-      const float r1 = (b1 ? part[3] : part[1]) + __shfl_xor_sync(0xffffffffu, b1 ? part[1] : part[3], 2);
-      const bool b0 = (k & 1) != 0;
-      float v = (b0 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b0 ? r0 : r1, 1);
+      // butterfly over the token's 8 lanes (slot j of lane k is head (k ^ j) & 3)
+      const float p0 = part2[0].x + part2[0].y, p1 = part2[1].x + part2[1].y;
+      const float p2 = part2[2].x + part2[2].y, p3 = part2[3].x + part2[3].y;
+      const float r0 = p0 + __shfl_xor_sync(0xffffffffu, p2, 2);
+      const float r1 = p1 + __shfl_xor_sync(0xffffffffu, p3, 2);
+      float v = r0 + __shfl_xor_sync(0xffffffffu, r1, 1);
       v += __shfl_xor_sync(0xffffffffu, v, 4);
       s_part[st] = v;
       if (k < 4) pxb[tt * kHeads + hk] = v;
     }
-    cluster.sync();   // the peer's partials of this tile have landed in xb
+    cluster_arrive_release();
+    bin_atomics();                      // previous tile, while the exchange completes
+    cluster_wait_acquire();             // the peer's partials of this tile are in xb
 
     // full scores (the same order of addition in both CTAs -> identical values)
     float s[C::kSteps];
@@ -238,68 +280,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
       const int tt = st * C::kSlots + sigma;
       const float other = xb[tt * kHeads + hk];
       const float v = rank == 0 ? s_part[st] + other : other + s_part[st];
-      s[st] = (t_tile + tt < t_end) ? v : -INFINITY;
+      s[st] = (FULL || t_tile + tt < t_end) ? v : -INFINITY;
       mx = fmaxf(mx, s[st]);
+      prev_valid[st] = FULL || t_tile + tt < t_end;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        vw[st][r] = *reinterpret_cast<const uint32_t*>(cb + (tt * R + r) * 16 + 8 + 4 * gh);
     }
+    // CTA-wide max per head: one barrier, then every warp reduces all warps' maxima
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     if (lane < kHeads) red[warp * kHeads + lane] = mx;
     __syncthreads();
-    if (tid < kHeads) {
-      float v = red[tid];
+    float mt = red[lane];                                   // entry lane: head lane & 3
 #pragma unroll
-      for (int w = 1; w < C::kWarps; ++w) v = fmaxf(v, red[w * kHeads + tid]);
-      mtile[tid] = v;
-    }
-    __syncthreads();
-    bool any_rescale = false;
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-      const float m_old = __shfl_sync(0xffffffffu, m_ref, hh);   // lane hh keeps head hh
-      any_rescale |= (m_old == -INFINITY) || (mtile[hh] > m_old + kRescaleSlack);
-    }
-    if (any_rescale) {   // uniform: every thread read the same mtile
-      const float m_new = (m_ref == -INFINITY || mtile[hk] > m_ref + kRescaleSlack) ? mtile[hk] : m_ref;
+    for (int e = 32; e < C::kWarps * kHeads; e += 32) mt = fmaxf(mt, red[e + lane]);
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));   // lane l: tile max of head l & 3 = hk
+    const bool raise = (m_ref == -INFINITY) || (mt > m_ref + kRescaleSlack);
+    if (__any_sync(0xffffffffu, raise)) {   // the same decision in every warp of the CTA
+      const float m_new = raise ? mt : m_ref;
       const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
       l_acc *= f;
       m_ref = m_new;
-      if (tid < kHeads) fh[tid] = f;   // thread tid < 4 is lane tid: head tid
-      __syncthreads();
+      if (tid < kHeads) fh[tid] = f;       // thread tid < 4 is lane tid: head tid
+      __syncthreads();                     // every atomic of the previous tile is done
       for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] *= fh[(i >> 3) & 3];
       __syncthreads();
     }
-    // weights: lanes with k < 4 exponentiate the first half of the steps, the others the
-    // second half; each lane then holds the weights of all steps of its token slot
-    float w[C::kSteps];
+    // weights of this tile (0 for tokens past the end); lanes k and k ^ 4 hold the same
+    // head, so only k < 4 adds to l
 #pragma unroll
     for (int st = 0; st < C::kSteps; ++st) {
-      const bool mine = (st < C::kSteps / 2) == (gh == 0);
-      float e = 0.f;
-      if (mine) {
-        e = exp2f(s[st] - m_ref);     // 0 for tokens past the end (s = -inf)
-        l_acc += e;
-      }
-      w[st] = e + __shfl_xor_sync(0xffffffffu, e, 4);
+      float e;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(s[st] - m_ref));
+      w[st] = e;
+      l_acc += (gh == 0) ? e : 0.f;
     }
-    // value-code bins: lane bins head hk for local groups 4 gh .. 4 gh + 3 (rotated by tau)
-#pragma unroll
-    for (int st = 0; st < C::kSteps; ++st) {
-      const int tt = st * C::kSlots + sigma;
-      if (t_tile + tt < t_end) {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint32_t word = *reinterpret_cast<const uint32_t*>(cb + (tt * R + r) * 16 + 8 + 4 * gh);
-          const uint32_t rot = __funnelshift_r(word, word, 8 * tau);   // byte i: group 4gh + ((i + tau) & 3)
-          float* bin_r = bins + r * (kCodes * kHeads * kLocalGroups) + hk * kLocalGroups + 4 * gh;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = (rot >> (8 * i)) & 0xff;
-            atomicAdd(bin_r + c * (kHeads * kLocalGroups) + ((i + tau) & 3), w[st]);
-          }
-        }
-      }
+  };
+
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int t_tile = t_begin + tile * kTile;
+    const int buf = tile & 1;
+    if (tile > 0) {
+      cp_async_wait_all();      // this tile's codes (issued one tile ago) have landed
+      __syncthreads();          // ... for every thread; the other buffer is free again
+    }
+    if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
+    if (t_tile + kTile <= t_end) {
+      run_tile(t_tile, buf, std::integral_constant<bool, true>());
+    } else {
+      run_tile(t_tile, buf, std::integral_constant<bool, false>());
     }
   }
+  bin_atomics();                // the last tile
 
   // ---- l: lanes hold disjoint shares of head hk; sum over slots, halves and warps ----
   l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 4);
