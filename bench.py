@@ -77,6 +77,24 @@ def recorded_traffic(workload: str, form: str):
     return float(rec["dram_bytes_per_launch"])
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank value over all ranks of the default process group (the value
+    itself when there is no group or a single rank)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms_per_step: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank per step and
+    the step takes ms_per_step on the slowest rank."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -263,11 +281,7 @@ def run_gpu(args):
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t.item())
+    total_ms_max = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms_max / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> decode -> host
@@ -306,11 +320,7 @@ def run_gpu(args):
         e2e_step()
     e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / n_e2e
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / n_e2e, dev)
 
     result = None
     if rank == 0:
@@ -321,7 +331,7 @@ def run_gpu(args):
         flops = algorithmic_flops(w, total_tokens)
         achieved_tflops = flops / (dec_mean_ms * 1e-3) / 1e12
         bytes_ = code_bytes(w, total_tokens)
-        value = world * total_tokens / (ms_per_step * 1e-3)
+        value = whole_job_rate(world, total_tokens, ms_per_step)
         result = {
             "metric": METRIC,
             "value": value,
@@ -351,7 +361,7 @@ def run_gpu(args):
                          "traffic_unit": "DRAM bytes per decode launch (ncu)",
                          "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {sm_max:.0f} MHz "
                                         f"(unit counts and max clock; HBM peak {pk_src})"},
-            "e2e": {"value": world * total_tokens / (e2e_ms * 1e-3), "unit": "KV tokens/s per layer",
+            "e2e": {"value": whole_job_rate(world, total_tokens, e2e_ms), "unit": "KV tokens/s per layer",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step,
             "clocks": clk.summary(),

@@ -154,7 +154,10 @@ int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
   const bool clustered = (s->n_q_heads / s->n_kv_heads) == 4;
   const long long units = static_cast<long long>(s->batch) * s->n_kv_heads * (clustered ? 2 : 1);
   const long long slots = static_cast<long long>(sm_count) * (clustered && s->R == 1 ? 2 : 1);
-  const long long max_splits = std::max(1LL, std::min(4096LL, (s->t_cap + 255LL) / 256LL));
+  // the clustered kernel amortizes a 64R KiB codebook load per CTA, so its splits stay
+  // >= 256 tokens; the plain kernel's splits may be as short as one 64-token block
+  const long long min_len = clustered ? 256LL : 64LL;
+  const long long max_splits = std::max(1LL, std::min(4096LL, (s->t_cap + min_len - 1) / min_len));
   for (long long n = 1; n <= max_splits; ++n) {
     const long long ctas = units * n;
     const long long waves = (ctas + slots - 1) / slots;

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
       }
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) s[hh] = 0.f;
-#pragma unroll 1
+#pragma unroll 4
       for (int G = 0; G < kGroups; ++G) {
         float kr[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
     const int G = dim / kVDims, d = dim % kVDims;
     const float* bh = bins + (hh * kGroups + G) * R * kCodes;
     float acc = 0.f;
+#pragma unroll 16
     for (int rc = 0; rc < R * kCodes; ++rc) {
       acc = fmaf(bh[rc], __ldg(vcb + (static_cast<size_t>(G) * R * kCodes + rc) * kVDims + d), acc);
     }
