@@ -238,14 +238,24 @@ def run_gpu(args):
                          host=d))
     total_tokens = int(sets[0]["host"]["seq_lens"].sum())
     shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base)
-    S = args.splits or cvq.suggest_splits(shape)
+    if args.splits:
+        S = args.splits
+    elif args.form == "naive":
+        # the naive attention runs one CTA per (split, KV head, sequence): ~4 waves of CTAs
+        S = max(1, min(4096, -(-4 * SM_COUNT_B200 // (w.batch * w.n_kv_heads)), w.t_cap // 64))
+    else:
+        S = cvq.suggest_splits(shape)
     parts = cvq.partials_alloc(shape, S, dev)
     out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
     ptab = (torch.empty((w.batch, w.n_q_heads, 16, w.R, 256, 4, 2), dtype=torch.float32, device=dev)
             if args.form == "table" else None)
+    if args.form == "naive":
+        kv_dims = (w.batch, w.n_kv_heads, w.t_cap, 128)
+        kh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
+        vh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 3 if args.form == "table" else 2
+    launches_per_step = 3 if args.form in ("table", "naive") else 2
 
     def step(i, ev=None):
         s = sets[i % n_sets]
@@ -255,6 +265,10 @@ def run_gpu(args):
             cvq.qtable(shape, s["q"], s["key_cb"], ptable=ptab)
             cvq.decode_attn(shape, ptab, s["key_codes"], s["val_codes"], s["seq_lens"], s["val_cb"],
                             S, partials=parts)
+        elif args.form == "naive":
+            cvq.naive_dequant(shape, s["key_cb"], s["val_cb"], s["key_codes"], s["val_codes"],
+                              s["seq_lens"], k_out=kh, v_out=vh)
+            cvq.naive_decode(shape, s["q"], kh, vh, s["seq_lens"], S, partials=parts)
         else:
             cvq.decode_attn_gqa(shape, s["q"], s["key_cb"], s["key_codes"], s["val_codes"],
                                 s["seq_lens"], s["val_cb"], S, partials=parts)
@@ -411,7 +425,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
-    ap.add_argument("--form", choices=["gqa", "table"], default="gqa")
+    ap.add_argument("--form", choices=["gqa", "table", "naive"], default="gqa",
+                    help="gqa: the library's fast path; table: the pages' per-query-head table "
+                         "form; naive: decode the cache to fp16 then attend (comparison path)")
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -22,7 +22,7 @@ from . import _binding as _b
 from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa: F401
 
 __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
-           "attend", "split_tokens", "suggest_splits", "partials_alloc", "CvqError"]
+           "attend", "naive_dequant", "naive_decode", "split_tokens", "suggest_splits", "partials_alloc", "CvqError"]
 
 
 def _ptr(t):
@@ -153,12 +153,44 @@ def combine(shape, n_splits, part_o, part_m, part_l, out=None, lse=None, stream=
     return out, lse
 
 
+def naive_dequant(shape, key_cb, val_cb, key_codes, val_codes, seq_lens, k_out=None, v_out=None,
+                  stream=None):
+    """The naive path's first half: every cached key (rotated by RoPE) and value decoded
+    into fp16 tensors [B, Hkv, t_cap, 128]."""
+    _require(key_cb, "key_cb", torch.float32)
+    _codes_check(key_codes, val_codes, seq_lens, val_cb)
+    dims = (shape.batch, shape.n_kv_heads, shape.t_cap, 128)
+    k_out = k_out if k_out is not None else torch.zeros(dims, dtype=torch.float16, device=key_codes.device)
+    v_out = v_out if v_out is not None else torch.zeros(dims, dtype=torch.float16, device=key_codes.device)
+    st = _b.lib.cvq_naive_dequant(ctypes.byref(shape), _ptr(key_cb), _head_stride(key_cb, "key"),
+                                  _ptr(key_codes), _ptr(val_codes), _ptr(seq_lens), _ptr(val_cb),
+                                  _head_stride(val_cb, "val"), _ptr(k_out), _ptr(v_out),
+                                  _stream(stream))
+    _b.check(st, "cvq_naive_dequant")
+    return k_out, v_out
+
+
+def naive_decode(shape, q, k, v, seq_lens, n_splits, partials=None, stream=None):
+    """The naive path's second half: split-T decode attention over fp16 keys / values."""
+    _require(q, "q", (torch.float32, torch.bfloat16))
+    _require(k, "k", torch.float16)
+    _require(v, "v", torch.float16)
+    _require(seq_lens, "seq_lens", torch.int32)
+    part_o, part_m, part_l = partials or partials_alloc(shape, n_splits, k.device)
+    st = _b.lib.cvq_naive_decode(ctypes.byref(shape), _ptr(q), _q_dtype(q), _ptr(k), _ptr(v),
+                                 _ptr(seq_lens), n_splits, _ptr(part_o), _ptr(part_m),
+                                 _ptr(part_l), _stream(stream))
+    _b.check(st, "cvq_naive_decode")
+    return part_o, part_m, part_l
+
+
 def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0, n_splits=None,
            form="gqa", stream=None):
     """One decode step: (out [B, Hq, 128], lse [B, Hq]) in fp32.
 
     form="gqa":   cvq_decode_attn_gqa + cvq_combine
     form="table": cvq_qtable + cvq_decode_attn + cvq_combine
+    form="naive": cvq_naive_dequant + cvq_naive_decode + cvq_combine (the comparison path)
     """
     shape = shape_of(q, key_codes, rope_base)
     if n_splits is None:
@@ -166,6 +198,9 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0
     if form == "table":
         P = qtable(shape, q, key_cb, stream=stream)
         parts = decode_attn(shape, P, key_codes, val_codes, seq_lens, val_cb, n_splits, stream=stream)
+    elif form == "naive":
+        kh, vh = naive_dequant(shape, key_cb, val_cb, key_codes, val_codes, seq_lens, stream=stream)
+        parts = naive_decode(shape, q, kh, vh, seq_lens, n_splits, stream=stream)
     elif form == "gqa":
         parts = decode_attn_gqa(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
                                 stream=stream)

@@ -51,6 +51,9 @@ def _load():
         "cvq_decode_attn_gqa": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P, P]),
         "cvq_combine": (I, [S, I, P, P, P, P, P, P]),
         "cvq_attend_static": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P]),
+        "cvq_naive_cache_bytes": (SZ, [S]),
+        "cvq_naive_dequant": (I, [S, P, I64, P, P, P, P, I64, P, P, P]),
+        "cvq_naive_decode": (I, [S, P, I, P, P, P, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -73,7 +76,8 @@ class _LazyLib:
 lib = _LazyLib()
 EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partials_bytes",
             "cvq_split_tokens", "cvq_suggest_splits", "cvq_qtable", "cvq_decode_attn",
-            "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static"]
+            "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static",
+            "cvq_naive_cache_bytes", "cvq_naive_dequant", "cvq_naive_decode"]
 
 
 def status_str(st: int) -> str:

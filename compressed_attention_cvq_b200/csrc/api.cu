@@ -233,4 +233,52 @@ cvq_status cvq_combine(const cvq_shape* s, int n_splits, const float* part_o, co
                                   static_cast<cudaStream_t>(stream)));
 }
 
+size_t cvq_naive_cache_bytes(const cvq_shape* s) {
+  if (check_shape(s) != CVQ_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->n_kv_heads * s->t_cap * kHeadDim * 2;
+}
+
+cvq_status cvq_naive_dequant(const cvq_shape* s, const float* key_cb, int64_t key_cb_head_stride,
+                             const uint8_t* key_codes, const uint8_t* val_codes,
+                             const int32_t* seq_lens, const float* val_cb,
+                             int64_t val_cb_head_stride, void* k_out, void* v_out, void* stream) {
+  CVQ_TRY(check_shape(s));
+  CVQ_TRY(check_ptr(key_cb));
+  CVQ_TRY(check_ptr(val_cb));
+  CVQ_TRY(check_ptr(key_codes));
+  CVQ_TRY(check_ptr(val_codes));
+  CVQ_TRY(check_ptr(k_out));
+  CVQ_TRY(check_ptr(v_out));
+  if (seq_lens == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0) return CVQ_ERR_ALIGN;
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
+  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s->R)));
+  PhaseTurns ph;
+  phase_turns_host(s->rope_base, &ph);
+  return from_cuda(launch_naive_dequant(*s, key_cb, key_cb_head_stride, val_cb, val_cb_head_stride,
+                                        key_codes, val_codes, seq_lens, ph, k_out, v_out,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+cvq_status cvq_naive_decode(const cvq_shape* s, const void* q, int q_dtype, const void* k,
+                            const void* v, const int32_t* seq_lens, int n_splits, float* part_o,
+                            float* part_m, float* part_l, void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
+  if (s->n_q_heads / s->n_kv_heads > 4) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_ptr(q));
+  CVQ_TRY(check_ptr(k));
+  CVQ_TRY(check_ptr(v));
+  if (seq_lens == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0) return CVQ_ERR_ALIGN;
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  CVQ_TRY(check_ptr(part_o));
+  if (part_m == nullptr || part_l == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(part_m) & 3u) || (reinterpret_cast<uintptr_t>(part_l) & 3u))
+    return CVQ_ERR_ALIGN;
+  return from_cuda(launch_naive_decode(*s, q, q_dtype, k, v, seq_lens, n_splits,
+                                       split_tokens_host(s->t_cap, n_splits), part_o, part_m,
+                                       part_l, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

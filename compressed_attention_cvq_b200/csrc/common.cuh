@@ -94,6 +94,16 @@ cudaError_t launch_decode_table(const cvq_shape& s, const DecodeArgs& a, cudaStr
 cudaError_t launch_decode_gqa(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
 // the clustered kernel for 4 query heads per KV head (decode_gqa.cu)
 cudaError_t launch_decode_gqa4(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+// the naive baseline (naive.cu, naive_decode.cu)
+cudaError_t launch_naive_dequant(const cvq_shape& s, const float* key_cb, long long key_stride,
+                                 const float* val_cb, long long val_stride,
+                                 const uint8_t* key_codes, const uint8_t* val_codes,
+                                 const int32_t* seq_lens, const PhaseTurns& phase, void* k_out,
+                                 void* v_out, cudaStream_t stream);
+cudaError_t launch_naive_decode(const cvq_shape& s, const void* q, int q_dtype, const void* k,
+                                const void* v, const int32_t* seq_lens, int n_splits,
+                                int split_tokens, float* part_o, float* part_m, float* part_l,
+                                cudaStream_t stream);
 cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
                            const float* part_m, const float* part_l, float* out, float* lse,
                            cudaStream_t stream);

@@ -167,6 +167,31 @@ CVQ_API cvq_status cvq_combine(const cvq_shape* shape, int n_splits, const float
                        void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * The naive path, for comparison (CommVQ summary page, "Key results": the optimized
+ * commutative-codebook implementation is measured against a naive implementation that
+ * decodes the cache before attending).  Not used by the calls above.
+ *
+ * cvq_naive_dequant -- decode every cached token into fp16 in HBM:
+ *   k_out[b, h, t, :] = RoPE_t(sum_r key codewords)  (keys rotated by position t),
+ *   v_out[b, h, t, :] = sum_r value codewords,       for t < seq_len[b];
+ *   k_out, v_out: [B, Hkv, t_cap, 128] fp16 (IEEE half bits), cvq_naive_cache_bytes() each;
+ *   entries t >= seq_len[b] are left untouched.  Other arguments as in cvq_decode_attn_gqa.
+ * cvq_naive_decode -- ordinary split-T decode attention over those fp16 keys and values
+ *   for every query head (Hq/Hkv <= 4); the same partial states as cvq_decode_attn (here m
+ *   is the exact split maximum); merge them with cvq_combine.
+ * ------------------------------------------------------------------------------- */
+CVQ_API size_t cvq_naive_cache_bytes(const cvq_shape* shape);
+CVQ_API cvq_status cvq_naive_dequant(const cvq_shape* shape, const float* key_cb,
+                                     int64_t key_cb_head_stride, const uint8_t* key_codes,
+                                     const uint8_t* val_codes, const int32_t* seq_lens,
+                                     const float* val_cb, int64_t val_cb_head_stride, void* k_out,
+                                     void* v_out, void* stream);
+CVQ_API cvq_status cvq_naive_decode(const cvq_shape* shape, const void* q, int q_dtype,
+                                    const void* k, const void* v, const int32_t* seq_lens,
+                                    int n_splits, float* part_o, float* part_m, float* part_l,
+                                    void* stream);
+
+/* ---------------------------------------------------------------------------------
  * cvq_attend_static -- cvq_decode_attn_gqa followed by cvq_combine, with the split
  * partial states kept in a fixed device array inside the library instead of memory
  * the caller allocates.  The paper has no counterpart: this is an interface for
