@@ -1,13 +1,17 @@
 """Benchmark: CommVQ decode attention, KV tokens/s per layer on B200.
 
-    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--form gqa|table]
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--form gqa|table|naive]
+                    [--append]
     python bench.py --impl reference ...     # the float64 CPU oracle, timed on host cores
 
 A step is one decode-attention pass over one layer of the workload: every query head
 of every sequence against its whole cached code stream (decode + combine; the table
 form adds the query-table build).  Inputs are resident in HBM before timing; 8
 independent layer-sized input sets rotate from step to step so no step finds the
-previous one's codes in L2 (8 x 36 MB > 126 MB L2 for the 128K layer).
+previous one's codes in L2 (8 x 36 MB > 126 MB L2 for the 128K layer).  With --append
+the step also writes the step's new key and value of every (sequence, KV head) into the
+code cache first (the write side: greedy residual encoding), at position seq_len - 1, so
+the cached length stays that of the workload.
 
 Printed: one JSON line (rank 0) with the metric, the decode kernel's roofline
 fraction (FP32 ALU bound), an end-to-end figure through host buffers, the clocks
@@ -56,6 +60,25 @@ def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
     codes = float(total_tokens) * w.n_kv_heads * 32 * w.R
     cbs = 2.0 * w.n_kv_heads * 16 * w.R * 256 * 8 * 4
     return codes + cbs
+
+
+def encode_work(w: workloads.Workload):
+    """Algorithmic work of one append (every sequence and KV head, key and value): per
+    group and round, 256 codewords x 8 dims x (sub, mul, add) FLOP; bytes = both codebooks
+    of every KV head + the new vectors + the written codes."""
+    units = w.batch * w.n_kv_heads
+    flops = float(units) * 2 * 16 * w.R * 256 * 8 * 3
+    bytes_ = 2.0 * w.n_kv_heads * 16 * w.R * 256 * 8 * 4 + units * (2 * 128 * 4 + 2 * 16 * w.R)
+    return flops, bytes_
+
+
+def append_summary(w: workloads.Workload, enc_ms):
+    """Timing of the append kernel inside the step, against its two bounds."""
+    flops, bytes_ = encode_work(w)
+    ms = statistics.mean(enc_ms)
+    return {"encode_ms": ms, "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
+            "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+            "achieved_gbs": bytes_ / (ms * 1e-3) / 1e9}
 
 
 def recorded_traffic(workload: str, form: str):
@@ -236,6 +259,10 @@ def run_gpu(args):
                          val_codes=torch.from_numpy(d["val_codes"]).to(dev),
                          seq_lens=torch.from_numpy(d["seq_lens"]).to(dev),
                          host=d))
+        if args.append:
+            nk, nv = workloads.new_tokens(w, layer=i)
+            sets[-1].update(new_k=torch.from_numpy(nk).to(dev), new_v=torch.from_numpy(nv).to(dev),
+                            pos=(sets[-1]["seq_lens"] - 1).contiguous(), host_new=(nk, nv))
     total_tokens = int(sets[0]["host"]["seq_lens"].sum())
     shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base)
     if args.splits:
@@ -255,12 +282,17 @@ def run_gpu(args):
         kh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
         vh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 3 if args.form in ("table", "naive") else 2
+    launches_per_step = (3 if args.form in ("table", "naive") else 2) + (1 if args.append else 0)
 
     def step(i, ev=None):
         s = sets[i % n_sets]
         if ev is not None:
             ev[0].record(stream)
+        if args.append:
+            cvq.encode_append(shape, s["new_k"], s["new_v"], s["key_cb"], s["val_cb"], s["pos"],
+                              s["key_codes"], s["val_codes"])
+        if ev is not None:
+            ev[3].record(stream)
         if args.form == "table":
             cvq.qtable(shape, s["q"], s["key_cb"], ptable=ptab)
             cvq.decode_attn(shape, ptab, s["key_codes"], s["val_codes"], s["seq_lens"], s["val_cb"],
@@ -281,7 +313,7 @@ def run_gpu(args):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -294,7 +326,8 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[3].elapsed_time(e[1]) for e in evs]
+    enc_ms = [e[0].elapsed_time(e[3]) for e in evs]
     total_ms_max = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms_max / args.steps
 
@@ -309,6 +342,10 @@ def run_gpu(args):
                    key_codes=torch.from_numpy(h["key_codes"]).pin_memory(),
                    val_codes=torch.from_numpy(h["val_codes"]).pin_memory(),
                    seq_lens=torch.from_numpy(h["seq_lens"]).pin_memory())
+    if args.append:
+        host_in.update(new_k=torch.from_numpy(sets[0]["host_new"][0]).pin_memory(),
+                       new_v=torch.from_numpy(sets[0]["host_new"][1]).pin_memory(),
+                       pos=torch.from_numpy(h["seq_lens"] - 1).pin_memory())
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
     host_out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory()
     host_lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32).pin_memory()
@@ -318,6 +355,10 @@ def run_gpu(args):
     def e2e_step():
         for k in dev_in:
             dev_in[k].copy_(host_in[k], non_blocking=True)
+        if args.append:
+            cvq.encode_append(shape, dev_in["new_k"], dev_in["new_v"], dev_in["key_cb"],
+                              dev_in["val_cb"], dev_in["pos"], dev_in["key_codes"],
+                              dev_in["val_codes"])
         o, l = cvq.attend(dev_in["q"], dev_in["key_cb"], dev_in["val_cb"], dev_in["key_codes"],
                           dev_in["val_codes"], dev_in["seq_lens"], w.rope_base, n_splits=S,
                           form=args.form)
@@ -362,6 +403,7 @@ def run_gpu(args):
             "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
                        "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R,
                        "q_dtype": w.q_dtype, "form": args.form, "n_splits": S,
+                       "append": bool(args.append),
                        "tokens_per_layer": total_tokens,
                        "l2": f"{N_INPUT_SETS} rotating layer input sets of "
                              f"{code_bytes(w, total_tokens) / 1e6:.0f} MB (> 126 MB L2 in total)",
@@ -378,6 +420,7 @@ def run_gpu(args):
             "e2e": {"value": whole_job_rate(world, total_tokens, e2e_ms), "unit": "KV tokens/s per layer",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step,
+            "append": append_summary(w, enc_ms) if args.append else None,
             "clocks": clk.summary(),
         }
     if world > 1:
@@ -429,6 +472,8 @@ def main(argv=None):
                     help="gqa: the library's fast path; table: the pages' per-query-head table "
                          "form; naive: decode the cache to fp16 then attend (comparison path)")
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--append", action="store_true",
+                    help="each step first encodes the step's new key/value into the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -22,7 +22,8 @@ from . import _binding as _b
 from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa: F401
 
 __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
-           "attend", "naive_dequant", "naive_decode", "split_tokens", "suggest_splits", "partials_alloc", "CvqError"]
+           "attend", "naive_dequant", "naive_decode", "encode_append", "split_tokens",
+           "suggest_splits", "partials_alloc", "CvqError"]
 
 
 def _ptr(t):
@@ -168,6 +169,24 @@ def naive_dequant(shape, key_cb, val_cb, key_codes, val_codes, seq_lens, k_out=N
                                   _stream(stream))
     _b.check(st, "cvq_naive_dequant")
     return k_out, v_out
+
+
+def encode_append(shape, keys, values, key_cb, val_cb, positions, key_codes, val_codes,
+                  stream=None):
+    """The write side of a decode step: codes of keys / values [B, Hkv, 128] (fp32,
+    pre-RoPE keys) written in place at [b, h, positions[b]] of key_codes / val_codes
+    [B, Hkv, t_cap, R, 16]; a position outside [0, t_cap) writes nothing."""
+    _require(keys, "keys", torch.float32)
+    _require(values, "values", torch.float32)
+    _require(key_cb, "key_cb", torch.float32)
+    _require(positions, "positions", torch.int32)
+    _codes_check(key_codes, val_codes, positions, val_cb)
+    st = _b.lib.cvq_encode_append(ctypes.byref(shape), _ptr(keys), _ptr(values), _ptr(key_cb),
+                                  _head_stride(key_cb, "key"), _ptr(val_cb),
+                                  _head_stride(val_cb, "val"), _ptr(positions),
+                                  _ptr(key_codes), _ptr(val_codes), _stream(stream))
+    _b.check(st, "cvq_encode_append")
+    return key_codes, val_codes
 
 
 def naive_decode(shape, q, k, v, seq_lens, n_splits, partials=None, stream=None):

@@ -54,6 +54,7 @@ def _load():
         "cvq_naive_cache_bytes": (SZ, [S]),
         "cvq_naive_dequant": (I, [S, P, I64, P, P, P, P, I64, P, P, P]),
         "cvq_naive_decode": (I, [S, P, I, P, P, P, I, P, P, P, P]),
+        "cvq_encode_append": (I, [S, P, P, P, I64, P, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -77,7 +78,8 @@ lib = _LazyLib()
 EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partials_bytes",
             "cvq_split_tokens", "cvq_suggest_splits", "cvq_qtable", "cvq_decode_attn",
             "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static",
-            "cvq_naive_cache_bytes", "cvq_naive_dequant", "cvq_naive_decode"]
+            "cvq_naive_cache_bytes", "cvq_naive_dequant", "cvq_naive_decode",
+            "cvq_encode_append"]
 
 
 def status_str(st: int) -> str:

@@ -281,4 +281,25 @@ cvq_status cvq_naive_decode(const cvq_shape* s, const void* q, int q_dtype, cons
                                        part_l, static_cast<cudaStream_t>(stream)));
 }
 
+cvq_status cvq_encode_append(const cvq_shape* s, const float* keys, const float* values,
+                             const float* key_cb, int64_t key_cb_head_stride, const float* val_cb,
+                             int64_t val_cb_head_stride, const int32_t* positions,
+                             uint8_t* key_codes, uint8_t* val_codes, void* stream) {
+  CVQ_TRY(check_shape(s));
+  CVQ_TRY(check_ptr(keys));
+  CVQ_TRY(check_ptr(values));
+  CVQ_TRY(check_ptr(key_cb));
+  CVQ_TRY(check_ptr(val_cb));
+  CVQ_TRY(check_ptr(key_codes));
+  CVQ_TRY(check_ptr(val_codes));
+  if (positions == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(positions) & 3u) != 0) return CVQ_ERR_ALIGN;
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
+  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s->R)));
+  if (s->t_cap == 0) return CVQ_OK;
+  return from_cuda(launch_encode_append(*s, keys, values, key_cb, key_cb_head_stride, val_cb,
+                                        val_cb_head_stride, positions, key_codes, val_codes,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

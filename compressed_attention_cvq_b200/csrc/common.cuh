@@ -104,6 +104,11 @@ cudaError_t launch_naive_decode(const cvq_shape& s, const void* q, int q_dtype, 
                                 const void* v, const int32_t* seq_lens, int n_splits,
                                 int split_tokens, float* part_o, float* part_m, float* part_l,
                                 cudaStream_t stream);
+// the write side: greedy residual encoding of one new key / value per (sequence, KV head)
+cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const float* values,
+                                 const float* key_cb, long long key_stride, const float* val_cb,
+                                 long long val_stride, const int32_t* positions,
+                                 uint8_t* key_codes, uint8_t* val_codes, cudaStream_t stream);
 cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
                            const float* part_m, const float* part_l, float* out, float* lse,
                            cudaStream_t stream);

@@ -192,6 +192,35 @@ CVQ_API cvq_status cvq_naive_decode(const cvq_shape* shape, const void* q, int q
                                     void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * cvq_encode_append -- the write side of a decode step: quantize one new key and one
+ * new value per (sequence, KV head) and store their codes at position positions[b] of
+ * the code cache.  The pages encode with a learned encoder (CommVQ abstract; summary
+ * page "Approach"), which needs trained weights; this call is the plain stand-in,
+ * greedy additive quantization (review page, "key_machinery": R residual rounds refine
+ * the reconstruction): for each group G and round r = 0..R-1 it picks the codeword
+ * nearest to the running residual and subtracts it.  The squared distance is summed
+ * in fp32 over the 8 dims in order 0..7 with no fused multiply-add; ties go to the
+ * smaller code.  Keys are encoded before RoPE (the cache holds pre-RoPE keys).
+ *
+ *   keys, values  [B, Hkv, 128] fp32 (16-byte aligned); a key group G is its pairs
+ *                 4G..4G+3 as dims 8G..8G+7 (re, im interleaved), a value group G is
+ *                 dims 8G..8G+7
+ *   key_cb, val_cb and their head strides as in cvq_decode_attn_gqa
+ *   positions     [B] int32 (device): the token index t each sequence writes; an index
+ *                 outside [0, t_cap) writes nothing for that sequence
+ *   key_codes, val_codes  [B, Hkv, t_cap, R, 16] uint8, written at [b, h, positions[b]]
+ *                 and nowhere else (the caller owns them; seq_lens is the caller's to
+ *                 advance)
+ *   Errors: CVQ_ERR_NULL / CVQ_ERR_ALIGN / CVQ_ERR_SHAPE / CVQ_ERR_UNSUPPORTED before any
+ *   launch; CVQ_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------------- */
+CVQ_API cvq_status cvq_encode_append(const cvq_shape* shape, const float* keys, const float* values,
+                                     const float* key_cb, int64_t key_cb_head_stride,
+                                     const float* val_cb, int64_t val_cb_head_stride,
+                                     const int32_t* positions, uint8_t* key_codes,
+                                     uint8_t* val_codes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * cvq_attend_static -- cvq_decode_attn_gqa followed by cvq_combine, with the split
  * partial states kept in a fixed device array inside the library instead of memory
  * the caller allocates.  The paper has no counterpart: this is an interface for

@@ -12,6 +12,7 @@ Layouts:
   key_codes  [B, Hkv, T_cap, R, 16]   uint8
   val_codes  [B, Hkv, T_cap, R, 16]   uint8
   seq_lens   [B]                      int32
+  new keys / values [B, Hkv, 128]     float32 (new_tokens: one decode step's append)
 
 Every tensor and every layer draws from its own stream of
 numpy.random.SeedSequence(seed).spawn(...), so workloads are reproducible bit for bit.
@@ -137,6 +138,17 @@ def generate(w: Workload, layer: int = 0, t_cap: int | None = None,
                 seq_lens=np.asarray(seq_lens, dtype=np.int32),
                 n_q_heads=Hq, n_kv_heads=Hkv, R=R, t_cap=T, batch=B,
                 rope_base=w.rope_base)
+
+
+def new_tokens(w: Workload, layer: int = 0, batch: int | None = None):
+    """One decode step's new keys and values [B, Hkv, 128] (float32, unit Gaussian: the
+    variance of a sum of R codewords of std sqrt(1/R)), as written to the cache by the
+    append call; pre-RoPE keys.  Their own seed stream, separate from generate()'s."""
+    B = batch if batch is not None else w.batch
+    s_k, s_v = np.random.SeedSequence([w.seed, layer, 1]).spawn(2)
+    shape = (B, w.n_kv_heads, 128)
+    return (np.random.default_rng(s_k).standard_normal(shape, dtype=np.float32),
+            np.random.default_rng(s_v).standard_normal(shape, dtype=np.float32))
 
 
 def small(batch=1, n_q_heads=4, n_kv_heads=1, t_cap=64, R=1, q_dtype="f32", cb_std=1.0,
