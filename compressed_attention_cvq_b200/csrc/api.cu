@@ -32,6 +32,7 @@ cvq_status check_shape(const cvq_shape* s) {
 cvq_status check_stride(int64_t stride, size_t per_head) {
   if (stride < 0) return CVQ_ERR_SHAPE;
   if (stride != 0 && static_cast<uint64_t>(stride) < per_head) return CVQ_ERR_SHAPE;
+  if (stride % 4 != 0) return CVQ_ERR_ALIGN;   // every head's codebook 16-byte aligned
   return CVQ_OK;
 }
 

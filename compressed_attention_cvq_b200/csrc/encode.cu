@@ -7,68 +7,90 @@
 // reconstruction) take the codeword nearest to the current residual and subtract it.
 // Keys are encoded before RoPE, as the cache stores them.
 //
-// One CTA per (sequence x KV head, group, key | value); thread c scores codeword c.  The
-// squared distance is summed in float32 in dim order 0..7 with no fused multiply-add, and
-// ties go to the smaller code, so the chosen code is a fixed function of the inputs.
+// One warp per (sequence x KV head, group, key | value); lane l scores codewords
+// l, l + 32, ..., l + 224.  The squared distance is summed in float32 in dim order 0..7
+// with no fused multiply-add, and ties go to the smaller code, so the chosen code is a
+// fixed function of the inputs.  No shared memory and no block barrier: the residual
+// lives in every lane's registers, and the winner's codeword reaches the warp by shuffles.
+// Every load of the first round (position, input, codewords) is independent of the others
+// and issued up front; the next round's codewords are loaded while this round's arg-min
+// runs.
 #include "common.cuh"
 
 namespace cvq {
 
 namespace {
 
-__global__ void __launch_bounds__(kCodes) encode_kernel(
+constexpr int kEncWarps = 8;                   // (group, key | value) units per CTA
+constexpr int kPerLane = kCodes / 32;          // codewords scored by each lane
+
+__device__ __forceinline__ void load_round(const float* cb_round, int lane, float4 (&w)[2 * kPerLane]) {
+  const float4* p = reinterpret_cast<const float4*>(cb_round) + 2 * lane;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    w[2 * i] = __ldg(p + 64 * i);
+    w[2 * i + 1] = __ldg(p + 64 * i + 1);
+  }
+}
+
+__global__ void __launch_bounds__(32 * kEncWarps) encode_kernel(
     const float* __restrict__ keys, const float* __restrict__ values,
     const float* __restrict__ key_cb, long long key_stride, const float* __restrict__ val_cb,
     long long val_stride, const int32_t* __restrict__ positions, uint8_t* __restrict__ key_codes,
     uint8_t* __restrict__ val_codes, int R, int n_kv_heads, int t_cap) {
-  __shared__ float res[8];
-  __shared__ float best_d[kCodes / 32];
-  __shared__ int best_c[kCodes / 32];
-  __shared__ int chosen;
-  const int bh = blockIdx.x, G = blockIdx.y, is_val = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const int unit = blockIdx.x * kEncWarps + (threadIdx.x >> 5);   // (bh, is_val, G)
+  const int G = unit & 15, is_val = (unit >> 4) & 1, bh = unit >> 5;
   const int b = bh / n_kv_heads, h = bh % n_kv_heads;
-  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
-  const int p = positions[b];
-  if (p < 0 || p >= t_cap) return;                       // uniform for the CTA
   const float* src = (is_val ? values : keys) + static_cast<size_t>(bh) * kHeadDim + 8 * G;
-  const float* cb = is_val ? val_cb + h * val_stride : key_cb + h * key_stride;
+  const float* cb = (is_val ? val_cb + h * val_stride : key_cb + h * key_stride) +
+                    static_cast<size_t>(G) * R * kCodes * 8;
+
+  float4 w[2 * kPerLane];
+  load_round(cb, lane, w);
+  const float4 x0 = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 x1 = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  const int p = positions[b];
+  if (p < 0 || p >= t_cap) return;                       // uniform for the warp
   uint8_t* out = (is_val ? val_codes : key_codes) +
                  ((static_cast<size_t>(bh) * t_cap + p) * R) * 16 + G;
-  if (c < 8) res[c] = src[c];
-  __syncthreads();
+  float res[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+
   for (int r = 0; r < R; ++r) {
-    const float4* cw = reinterpret_cast<const float4*>(cb + ((static_cast<size_t>(G) * R + r) * kCodes + c) * 8);
-    const float4 lo = __ldg(cw), hi = __ldg(cw + 1);
-    const float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    float acc = 0.f;
+    // this lane's nearest codeword (scanned in ascending code order, strict <)
+    float bd = INFINITY;
+    int bi = 0;
+    float bw[8];
 #pragma unroll
-    for (int d = 0; d < 8; ++d) {
-      const float diff = __fsub_rn(res[d], w[d]);
-      acc = __fadd_rn(acc, __fmul_rn(diff, diff));
+    for (int i = 0; i < kPerLane; ++i) {
+      const float c[8] = {w[2 * i].x, w[2 * i].y, w[2 * i].z, w[2 * i].w,
+                          w[2 * i + 1].x, w[2 * i + 1].y, w[2 * i + 1].z, w[2 * i + 1].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        const float diff = __fsub_rn(res[d], c[d]);
+        acc = __fadd_rn(acc, __fmul_rn(diff, diff));
+      }
+      const bool better = (i == 0) || (acc < bd);
+      bd = better ? acc : bd;
+      bi = better ? i : bi;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) bw[d] = better ? c[d] : bw[d];
     }
-    // arg-min over the 256 codewords, smaller code on ties
-    float bd = acc;
-    int bc = c;
+    if (r + 1 < R) load_round(cb + static_cast<size_t>(r + 1) * kCodes * 8, lane, w);
+    // warp arg-min over (distance, code); code = lane + 32 * i
+    float md = bd;
+    int mc = lane + 32 * bi;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float od = __shfl_xor_sync(0xffffffffu, bd, o);
-      const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
-      if (od < bd || (od == bd && oc < bc)) { bd = od; bc = oc; }
+      const float od = __shfl_xor_sync(0xffffffffu, md, o);
+      const int oc = __shfl_xor_sync(0xffffffffu, mc, o);
+      if (od < md || (od == md && oc < mc)) { md = od; mc = oc; }
     }
-    if (lane == 0) { best_d[warp] = bd; best_c[warp] = bc; }
-    __syncthreads();
-    if (c == 0) {
-      float d0 = best_d[0];
-      int c0 = best_c[0];
-      for (int i = 1; i < kCodes / 32; ++i) {
-        if (best_d[i] < d0 || (best_d[i] == d0 && best_c[i] < c0)) { d0 = best_d[i]; c0 = best_c[i]; }
-      }
-      chosen = c0;
-      out[r * 16] = static_cast<uint8_t>(c0);
-    }
-    __syncthreads();
-    if (c < 8) res[c] = __fsub_rn(res[c], cb[((static_cast<size_t>(G) * R + r) * kCodes + chosen) * 8 + c]);
-    __syncthreads();
+    if (lane == 0) out[r * 16] = static_cast<uint8_t>(mc);
+    // residual -= the chosen codeword, held by lane mc & 31
+#pragma unroll
+    for (int d = 0; d < 8; ++d) res[d] = __fsub_rn(res[d], __shfl_sync(0xffffffffu, bw[d], mc & 31));
   }
 }
 
@@ -78,10 +100,11 @@ cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const fl
                                  const float* key_cb, long long key_stride, const float* val_cb,
                                  long long val_stride, const int32_t* positions,
                                  uint8_t* key_codes, uint8_t* val_codes, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(s.batch) * s.n_kv_heads, kGroups, 2);
-  encode_kernel<<<grid, kCodes, 0, stream>>>(keys, values, key_cb, key_stride, val_cb, val_stride,
-                                             positions, key_codes, val_codes, s.R, s.n_kv_heads,
-                                             s.t_cap);
+  // units = B * Hkv * 2 * 16, a multiple of kEncWarps
+  const unsigned blocks = static_cast<unsigned>(s.batch) * s.n_kv_heads * 32 / kEncWarps;
+  encode_kernel<<<blocks, 32 * kEncWarps, 0, stream>>>(keys, values, key_cb, key_stride, val_cb,
+                                                        val_stride, positions, key_codes, val_codes,
+                                                        s.R, s.n_kv_heads, s.t_cap);
   return cudaGetLastError();
 }
 

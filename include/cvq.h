@@ -54,7 +54,7 @@ typedef enum {
   CVQ_OK = 0,
   CVQ_ERR_NULL = 1,        /* a required pointer is NULL                            */
   CVQ_ERR_SHAPE = 2,       /* inconsistent or out-of-range sizes                    */
-  CVQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                      */
+  CVQ_ERR_ALIGN = 3,       /* a pointer (or a codebook head stride) is not 16-byte aligned */
   CVQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (head_dim != 128, R > 2 ...) */
   CVQ_ERR_WORKSPACE = 5,   /* n_splits out of range                                 */
   CVQ_ERR_CUDA = 6,        /* the CUDA runtime reported an error                    */
@@ -91,7 +91,8 @@ CVQ_API int cvq_abi_version(void);
  *   q        [B, Hq, 128]           fp32 or bf16 (q_dtype), the already-rotated query
  *   key_cb   [Hkv][16, R, 256, 4, 2] fp32; KV head h starts at key_cb + h * key_cb_head_stride
  *            (stride in floats; 0 = one codebook shared by all KV heads, otherwise
- *            >= 16*R*256*8)
+ *            >= 16*R*256*8; a multiple of 4 so every head starts 16-byte aligned, else
+ *            CVQ_ERR_ALIGN)
  *   ptable   [B, Hq, 16, R, 256, 4, 2] fp32 output, cvq_ptable_bytes(shape) bytes
  * ------------------------------------------------------------------------------- */
 CVQ_API size_t cvq_ptable_bytes(const cvq_shape* shape);
@@ -130,7 +131,7 @@ CVQ_API int cvq_suggest_splits(const cvq_shape* shape, int sm_count);
  *   val_codes  [B, Hkv, t_cap, R, 16] uint8
  *   seq_lens   [B] int32 (device)
  *   val_cb     [Hkv][16, R, 256, 8] fp32, KV head h at val_cb + h * val_cb_head_stride
- *              (0 = shared, otherwise >= 16*R*256*8)
+ *              (0 = shared, otherwise >= 16*R*256*8 and a multiple of 4)
  *   part_*     split partial states, see above
  * ------------------------------------------------------------------------------- */
 CVQ_API cvq_status cvq_decode_attn(const cvq_shape* shape, const float* ptable, const uint8_t* key_codes,

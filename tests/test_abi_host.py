@@ -1,7 +1,7 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports every
 entry point include/cvq.h declares, reports sizes, and rejects bad arguments with a
 status before launching anything.  Every call below carries at least one invalid
-argument, so none of them reaches a kernel launch."""
+argument or has nothing to do (t_cap = 0), so none of them reaches a kernel launch."""
 import ctypes
 import os
 import re
@@ -92,6 +92,7 @@ def test_qtable_errors():
     assert _qtable(_shape(rope_base=1.0)) == 2
     assert _qtable(_shape(), stride=-5) == 2
     assert _qtable(_shape(), stride=100) == 2                     # below one head's size
+    assert _qtable(_shape(), stride=65536 + 2) == 3               # heads not 16-byte aligned
 
 
 def _decode(shape, n_splits=4, **kw):
@@ -160,3 +161,24 @@ def test_product_never_touches_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"\boracle\b", src), fn
+
+
+def _encode(shape, **kw):
+    a = dict(k=FAKE, v=FAKE, kcb=FAKE, kstride=0, vcb=FAKE, vstride=0, pos=FAKE, kc=FAKE, vc=FAKE)
+    a.update(kw)
+    return b.lib.cvq_encode_append(ctypes.byref(shape) if shape is not None else None, a["k"],
+                                   a["v"], a["kcb"], a["kstride"], a["vcb"], a["vstride"],
+                                   a["pos"], a["kc"], a["vc"], None)
+
+
+def test_encode_append_errors():
+    s = _shape()
+    assert _encode(None) == 1
+    assert _encode(s, k=None) == 1
+    assert _encode(s, v=MISALIGNED) == 3
+    assert _encode(s, pos=None) == 1
+    assert _encode(s, kc=MISALIGNED) == 3
+    assert _encode(s, vstride=16) == 2
+    assert _encode(s, kstride=65536 + 1) == 3
+    assert _encode(_shape(R=3)) == 4
+    assert _encode(_shape(t_cap=0)) == 0           # nothing to write, no launch
