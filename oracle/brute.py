@@ -6,13 +6,14 @@ the NumPy oracle: the two must agree to ~1e-12.
 
 The definition followed is the same (CommVQ review page, pith.science arXiv
 2506.18879, "key_machinery"; CommVQ abstract on the aitopics.org page):
-  key dim (2j + e), e in {0, 1}, pair j, group G = j // 4, slot p = j % 4:
+  key dim (2j + e), e in {0, 1}, pair j, group G = j // PPG, slot p = j % PPG
+  (PPG pairs per group: 4 with 256-entry codebooks, 32 in the paper's 64-entry layout):
       k = sum_r key_cb[h][G][r][code][p][e]
   RoPE at position t, angle a = base^(-2j/128) * t:
       k'[2j]   = cos(a) k[2j] - sin(a) k[2j+1]
       k'[2j+1] = sin(a) k[2j] + cos(a) k[2j+1]
   s_t = sum_d q[d] k'[d] / sqrt(128)
-  out[d] = sum_t softmax(s)_t * v_t[d],   v_t[8G + d] = sum_r val_cb[h][G][r][code][d]
+  out[d] = sum_t softmax(s)_t * v_t[d],   v_t[VD G + d] = sum_r val_cb[h][G][r][code][d]
 """
 from __future__ import annotations
 
@@ -26,13 +27,15 @@ def brute_attend_head(q, key_cb_h, val_cb_h, key_codes, val_codes, seq_len, base
     if seq_len == 0:
         return [0.0] * 128, -math.inf
     R = len(key_codes[0])
+    ppg = len(key_cb_h[0][0][0])      # pairs per key group
+    vd = len(val_cb_h[0][0][0])       # dims per value group
     s = []
     vals = []
     for t in range(seq_len):
         key = [0.0] * 128
         for d in range(128):
             j, e = divmod(d, 2)
-            G, p = divmod(j, 4)
+            G, p = divmod(j, ppg)
             acc = 0.0
             for r in range(R):
                 acc += float(key_cb_h[G][r][int(key_codes[t][r][G])][p][e])
@@ -47,7 +50,7 @@ def brute_attend_head(q, key_cb_h, val_cb_h, key_codes, val_codes, seq_len, base
         s.append(dot / math.sqrt(128.0))
         v = [0.0] * 128
         for d in range(128):
-            G, dd = divmod(d, 8)
+            G, dd = divmod(d, vd)
             acc = 0.0
             for r in range(R):
                 acc += float(val_cb_h[G][r][int(val_codes[t][r][G])][dd])

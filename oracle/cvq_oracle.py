@@ -10,7 +10,7 @@ definition states):
 
   1. theta_j = base^(-2j/128), j = 0..63 (RoPE frequencies of 64 interleaved pairs).
   2. Each cached key is reconstructed *before* RoPE as an additive sum of R key
-     codewords per group of 4 pairs.  A key codeword is the commutative 2x2 block
+     codewords per group of PPG pairs (layouts below).  A key codeword is the commutative 2x2 block
      [[a,-b],[b,a]]; applied to e_1 it gives the pair value (a, b).
      -- CommVQ review page (pith.science, arXiv 2506.18879), "key_machinery":
         per-subspace codebook matrices [[x, y], [-y, x]] that commute with the RoPE
@@ -19,7 +19,7 @@ definition states):
      position t.
   4. score_t = q . RoPE_t(k_t) / sqrt(128), q being the already-rotated query.
   5. Softmax with max subtraction; lse = m + ln(sum exp(s - m)).
-  6. Each value is reconstructed as an additive sum of R codewords per group of 8
+  6. Each value is reconstructed as an additive sum of R codewords per group of VD
      dims ("decoded via simple matrix multiplication" -- CommVQ abstract, on the
      aitopics.org "1-bit quantization" page), and out = sum_t w_t v_t.
 
@@ -37,12 +37,19 @@ Also here, each following the same pages:
 
 Layouts (all row-major):
   q          [B, Hq, 128]                 pair j = dims (2j, 2j+1)
-  key_cb     [Hkv, 16, R, 256, 4, 2]       (group G, round r, code c, pair p, re/im)
-  val_cb     [Hkv, 16, R, 256, 8]          (group G, round r, code c, dim d)
-  key_codes  [B, Hkv, T_cap, R, 16] uint8
-  val_codes  [B, Hkv, T_cap, R, 16] uint8
+  key_cb     [Hkv, NG, R, NC, PPG, 2]      (group G, round r, code c, pair p, re/im)
+  val_cb     [Hkv, NG, R, NC, VD]          (group G, round r, code c, dim d)
+  key_codes  [B, Hkv, T_cap, R, NG] uint8  (token-major; attend() also takes the
+  val_codes  [B, Hkv, T_cap, R, NG] uint8   planar order [B, Hkv, NG, R, T_cap])
   seq_lens   [B] int
-Query head hq reads KV head hq // (Hq // Hkv).
+Query head hq reads KV head hq // (Hq // Hkv).  A group G is PPG consecutive RoPE
+pairs of the key (pairs PPG*G .. PPG*G + PPG - 1) and VD = 2*PPG consecutive dims of
+the value ("consecutive sub-vectors share one quantized index (group size g)" --
+review page, "key_machinery").  Two instances are used, read off the codebook shapes:
+  g = 8 scalars:  NG = 16, PPG = 4,  NC = 256 codewords, R = 1 or 2 (1 or 2 bits);
+  g = 64 scalars: NG = 2,  PPG = 32, NC = 64 codewords,  R = 11 or 21 -- the paper's own
+                  parameterization, R log2(64) / 64 = 1.03 or 1.97 bits (CommVQ summary
+                  page, "Key results" and "Limitations").
 """
 from __future__ import annotations
 
@@ -72,28 +79,32 @@ def rope_theta(base: float) -> np.ndarray:
 # step 2 / 6: additive codebook reconstruction
 # ---------------------------------------------------------------------------
 def decode_keys(key_cb_h: np.ndarray, codes: np.ndarray) -> np.ndarray:
-    """Pre-RoPE keys [T, 128] from codes [T, R, 16] and one head's codebook
-    [16, R, 256, 4, 2].  Pair j = 4G + p holds sum_r key_cb[G, r, code[r, G], p]."""
+    """Pre-RoPE keys [T, 128] from codes [T, R, NG] and one head's codebook
+    [NG, R, NC, PPG, 2].  Pair j = PPG*G + p holds sum_r key_cb[G, r, code[r, G], p]."""
     codes = np.asarray(codes)
     T, R, _ = codes.shape
     cb = np.asarray(key_cb_h, dtype=np.float64)
-    k = np.zeros((T, N_GROUPS, PAIRS_PER_GROUP, 2), dtype=np.float64)
+    n_groups, ppg = cb.shape[0], cb.shape[3]
+    assert n_groups * ppg == N_PAIRS and codes.shape[2] == n_groups
+    k = np.zeros((T, n_groups, ppg, 2), dtype=np.float64)
     for r in range(R):
-        for g in range(N_GROUPS):
+        for g in range(n_groups):
             k[:, g] += cb[g, r][codes[:, r, g]]
-    # [T, G, p, (re, im)] -> dim 8G + 2p + comp = 2j + comp with j = 4G + p
+    # [T, G, p, (re, im)] -> dim 2 PPG G + 2p + comp = 2j + comp with j = PPG G + p
     return k.reshape(T, HEAD_DIM)
 
 
 def decode_values(val_cb_h: np.ndarray, codes: np.ndarray) -> np.ndarray:
-    """Values [T, 128] from codes [T, R, 16] and one head's codebook [16, R, 256, 8].
-    Dim 8G + d holds sum_r val_cb[G, r, code[r, G], d]."""
+    """Values [T, 128] from codes [T, R, NG] and one head's codebook [NG, R, NC, VD].
+    Dim VD*G + d holds sum_r val_cb[G, r, code[r, G], d]."""
     codes = np.asarray(codes)
     T, R, _ = codes.shape
     cb = np.asarray(val_cb_h, dtype=np.float64)
-    v = np.zeros((T, N_GROUPS, VDIMS_PER_GROUP), dtype=np.float64)
+    n_groups, vd = cb.shape[0], cb.shape[3]
+    assert n_groups * vd == HEAD_DIM and codes.shape[2] == n_groups
+    v = np.zeros((T, n_groups, vd), dtype=np.float64)
     for r in range(R):
-        for g in range(N_GROUPS):
+        for g in range(n_groups):
             v[:, g] += cb[g, r][codes[:, r, g]]
     return v.reshape(T, HEAD_DIM)
 
@@ -159,11 +170,21 @@ def attend_head(q_vec, key_cb_h, val_cb_h, key_codes_bh, val_codes_bh, seq_len, 
     return out, lse
 
 
-def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, base, heads=None):
+def token_major(codes):
+    """Planar codes [B, Hkv, NG, R, T] viewed token-major [B, Hkv, T, R, NG] (a
+    transposed view; no value changes)."""
+    return np.transpose(np.asarray(codes), (0, 1, 4, 3, 2))
+
+
+def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, base, heads=None,
+           codes_layout="token"):
     """Full decode step.  Returns out [B, Hq, 128] and lse [B, Hq] (float64).
 
     `heads`, if given, is an iterable of (b, hq) to compute; other entries are NaN.
+    `codes_layout` "planar" takes codes as [B, Hkv, NG, R, T_cap].
     """
+    if codes_layout == "planar":
+        key_codes, val_codes = token_major(key_codes), token_major(val_codes)
     q = np.asarray(q, dtype=np.float64)
     B, Hq, _ = q.shape
     Hkv = key_codes.shape[1]
@@ -183,17 +204,17 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, base, heads=None):
 # ---------------------------------------------------------------------------
 def qtable(q, key_cb, n_kv_heads):
     """P[b, hq, G, r, c, p, (re, im)] = conj(q_j) * c with q_j = q[2j] + i q[2j+1],
-    c = a + i b the codeword of KV head hq // (Hq/Hkv), j = 4G + p."""
+    c = a + i b the codeword of KV head hq // (Hq/Hkv), j = PPG*G + p."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, _ = q.shape
     cb = np.asarray(key_cb, dtype=np.float64)
-    R = cb.shape[2]
-    P = np.empty((B, Hq, N_GROUPS, R, N_CODES, PAIRS_PER_GROUP, 2))
+    n_groups, R, n_codes, ppg = cb.shape[1], cb.shape[2], cb.shape[3], cb.shape[4]
+    P = np.empty((B, Hq, n_groups, R, n_codes, ppg, 2))
     for b in range(B):
         for hq in range(Hq):
             h = kv_head_of(hq, Hq, n_kv_heads)
-            qc = (q[b, hq, 0::2] - 1j * q[b, hq, 1::2]).reshape(N_GROUPS, 1, 1, PAIRS_PER_GROUP)
-            c = cb[h, ..., 0] + 1j * cb[h, ..., 1]          # [16, R, 256, 4]
+            qc = (q[b, hq, 0::2] - 1j * q[b, hq, 1::2]).reshape(n_groups, 1, 1, ppg)
+            c = cb[h, ..., 0] + 1j * cb[h, ..., 1]          # [NG, R, NC, PPG]
             prod = qc * c
             P[b, hq, ..., 0] = prod.real
             P[b, hq, ..., 1] = prod.imag
@@ -201,15 +222,16 @@ def qtable(q, key_cb, n_kv_heads):
 
 
 def score_from_table(P_bh, key_codes_bh, seq_len, base):
-    """score_t = sum_{G,p} Re(e^{i theta_{4G+p} t} * sum_r P[G, r, code_{t,r,G}, p]) / sqrt(128)."""
+    """score_t = sum_{G,p} Re(e^{i theta_{PPG G+p} t} * sum_r P[G, r, code_{t,r,G}, p]) / sqrt(128)."""
     theta = rope_theta(base)
     T = seq_len
     codes = key_codes_bh[:T]
     R = codes.shape[1]
-    z = np.zeros((T, N_GROUPS, PAIRS_PER_GROUP), dtype=np.complex128)
+    n_groups, ppg = P_bh.shape[0], P_bh.shape[3]
+    z = np.zeros((T, n_groups, ppg), dtype=np.complex128)
     for r in range(R):
-        for g in range(N_GROUPS):
-            ent = P_bh[g, r][codes[:, r, g]]               # [T, 4, 2]
+        for g in range(n_groups):
+            ent = P_bh[g, r][codes[:, r, g]]               # [T, PPG, 2]
             z[:, g] += ent[..., 0] + 1j * ent[..., 1]
     phase = np.exp(1j * np.arange(T, dtype=np.float64)[:, None] * theta[None, :])
     return np.real(phase * z.reshape(T, N_PAIRS)).sum(axis=1) * SCALE
@@ -218,21 +240,21 @@ def score_from_table(P_bh, key_codes_bh, seq_len, base):
 # ---------------------------------------------------------------------------
 # the method's value reorder: probability bins times the value codebook
 # ---------------------------------------------------------------------------
-def value_bins(w, val_codes_bh):
+def value_bins(w, val_codes_bh, n_codes=N_CODES):
     """bins[G, r, c] = sum_t w_t [val_code_{t,r,G} == c]."""
     w = np.asarray(w, dtype=np.float64)
     T = w.shape[0]
     codes = val_codes_bh[:T]
-    R = codes.shape[1]
-    bins = np.zeros((N_GROUPS, R, N_CODES))
+    R, n_groups = codes.shape[1], codes.shape[2]
+    bins = np.zeros((n_groups, R, n_codes))
     for r in range(R):
-        for g in range(N_GROUPS):
+        for g in range(n_groups):
             np.add.at(bins[g, r], codes[:, r, g], w)
     return bins
 
 
 def output_from_bins(bins, val_cb_h):
-    """out[8G + d] = sum_{r, c} bins[G, r, c] * val_cb[G, r, c, d]."""
+    """out[VD*G + d] = sum_{r, c} bins[G, r, c] * val_cb[G, r, c, d]."""
     cb = np.asarray(val_cb_h, dtype=np.float64)
     out = np.einsum("grc,grcd->gd", bins, cb)
     return out.reshape(HEAD_DIM)
@@ -275,10 +297,10 @@ def combine(m, l, o):
 # ---------------------------------------------------------------------------
 # size accounting of the cache layout
 # ---------------------------------------------------------------------------
-def code_bytes_per_token(R: int) -> int:
+def code_bytes_per_token(R: int, n_groups: int = N_GROUPS) -> int:
     """Bytes of key + value codes one token of one KV head occupies:
-    one uint8 per (group, round), 16 groups, for keys and again for values."""
-    return 2 * R * N_GROUPS
+    one uint8 per (group, round), for keys and again for values."""
+    return 2 * R * n_groups
 
 
 def fp16_kv_bytes_per_token() -> int:

@@ -307,6 +307,93 @@ def test_instance_is_one_and_two_bits():
 
 
 # ---------------------------------------------------------------------------
+# 9. the paper's own parameterization: 64-entry codebooks over groups of 64 scalars
+#    (32 consecutive RoPE pairs share one index), R = 11 / 21 (CommVQ summary page,
+#    "Key results" and "Limitations"; review page "key_machinery")
+# ---------------------------------------------------------------------------
+def _wide_case(T=6, R=3, Hq=2, Hkv=1, seed=0):
+    return workloads.small(batch=1, n_q_heads=Hq, n_kv_heads=Hkv, t_cap=T, R=R, seed=seed,
+                           cb_std=math.sqrt(1.0 / R), group_dim=64)
+
+
+@pytest.mark.parametrize("T,R,Hq,Hkv,seed", [(1, 1, 1, 1, 40), (5, 3, 2, 1, 41), (8, 11, 4, 2, 42),
+                                             (3, 21, 2, 1, 43)])
+def test_wide_brute_force_agrees(T, R, Hq, Hkv, seed):
+    d = _wide_case(T=T, R=R, Hq=Hq, Hkv=Hkv, seed=seed)
+    assert d["key_codes"].shape == (1, Hkv, 2, R, T) and int(d["key_codes"].max()) < 64
+    out, lse = O.attend(d["q"], d["key_cb"], d["val_cb"], d["key_codes"], d["val_codes"],
+                        d["seq_lens"], d["rope_base"], codes_layout="planar")
+    for hq in range(Hq):
+        h = O.kv_head_of(hq, Hq, Hkv)
+        # planar [G, r, t] -> nested [t][r][G], by explicit loops
+        kcodes = [[[int(d["key_codes"][0, h, G, r, t]) for G in range(2)] for r in range(R)]
+                  for t in range(T)]
+        vcodes = [[[int(d["val_codes"][0, h, G, r, t]) for G in range(2)] for r in range(R)]
+                  for t in range(T)]
+        bo, bl = brute.brute_attend_head(d["q"][0, hq].tolist(), d["key_cb"][h], d["val_cb"][h],
+                                         kcodes, vcodes, T, d["rope_base"])
+        np.testing.assert_allclose(out[0, hq], bo, rtol=0, atol=1e-12)
+        assert abs(lse[0, hq] - bl) <= 1e-12
+
+
+def test_wide_closed_form_groups_and_rounds():
+    """Every code 5 (keys) / 7 (values); key codeword entry of group G, round r, pair slot
+    p = (100 (G+1) + p + 1) (r + 1) (1, -1), so pair j = 32 G + p of the decoded key is
+    (100 (G+1) + p + 1) R (R+1)/2 (1, -1); value entry (1000 G + d) 2^-r, so value dim
+    64 G + d is (1000 G + d)(2 - 2^(1-R))."""
+    R = 11
+    kc = np.zeros((2, R, 64, 32, 2))
+    vc = np.zeros((2, R, 64, 64))
+    for G in range(2):
+        for r in range(R):
+            for p in range(32):
+                kc[G, r, 5, p] = np.array([1.0, -1.0]) * (100 * (G + 1) + p + 1) * (r + 1)
+            vc[G, r, 7] = (1000.0 * G + np.arange(64)) * 2.0 ** -r
+    k = O.decode_keys(kc, np.full((1, R, 2), 5))
+    v = O.decode_values(vc, np.full((1, R, 2), 7))
+    for j in range(64):
+        G, p = divmod(j, 32)
+        e = (100 * (G + 1) + p + 1) * R * (R + 1) / 2
+        assert k[0, 2 * j] == e and k[0, 2 * j + 1] == -e
+    for dd in range(128):
+        G, d = divmod(dd, 64)
+        assert abs(v[0, dd] - (1000 * G + d) * (2 - 2.0 ** (1 - R))) < 1e-9
+
+
+def test_wide_table_form_equals_reconstruct_form():
+    d = _wide_case(T=700, R=11, Hq=4, Hkv=1, seed=44)
+    kt = O.token_major(d["key_codes"])
+    P = O.qtable(d["q"], d["key_cb"], 1)
+    assert P.shape == (1, 4, 2, 11, 64, 32, 2)
+    for hq in range(4):
+        a = O.score_from_table(P[0, hq], kt[0, 0], 700, d["rope_base"])
+        b = O.scores(d["q"][0, hq], d["key_cb"][0], kt[0, 0], 700, d["rope_base"])
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_wide_value_reorder_identity():
+    d = _wide_case(T=900, R=21, Hq=1, seed=45)
+    kt, vt = O.token_major(d["key_codes"]), O.token_major(d["val_codes"])
+    s = O.scores(d["q"][0, 0], d["key_cb"][0], kt[0, 0], 900, d["rope_base"])
+    w, _ = O.softmax_weights(s)
+    direct = w @ O.decode_values(d["val_cb"][0], vt[0, 0])
+    bins = O.value_bins(w, vt[0, 0], n_codes=64)
+    assert bins.shape == (2, 21, 64)
+    np.testing.assert_allclose(O.output_from_bins(bins, d["val_cb"][0]), direct, atol=1e-12)
+    assert abs(bins.sum() - 2 * 21) < 1e-12
+
+
+def test_wide_sizes():
+    """R = 11 / 21 with 64 codewords over 64-scalar groups: R log2(64) / 64 bits per scalar
+    (1.03 / 1.97); one uint8 per (group, round) is 2 R bytes per token for keys and again
+    for values."""
+    assert O.avg_bits(11, 64, 64) == 66 / 64 and O.avg_bits(21, 64, 64) == 126 / 64
+    assert O.code_bytes_per_token(11, n_groups=2) == 44
+    d = _wide_case(T=4, R=11)
+    assert d["key_codes"][0, 0, :, :, 0].nbytes * 2 == O.code_bytes_per_token(11, n_groups=2)
+
+
+# ---------------------------------------------------------------------------
 # planted mistakes: each must make at least one pin above fail
 # ---------------------------------------------------------------------------
 def _pins_pass():
@@ -318,6 +405,9 @@ def _pins_pass():
         test_table_form_equals_reconstruct_form(2)
         test_value_reorder_identity(2, "zipf1.1")
         test_rope_is_complex_multiplication()
+        test_wide_brute_force_agrees(8, 11, 4, 2, 42)
+        test_wide_closed_form_groups_and_rounds()
+        test_wide_value_reorder_identity()
     except AssertionError:
         return False
     return True
@@ -355,14 +445,29 @@ def _bad_decode_values(val_cb_h, codes):       # transposed (G, d) inside the va
     return v.reshape(-1, 16, 8).transpose(0, 2, 1).reshape(-1, 128)
 
 
+def _bad_decode_keys_strided(key_cb_h, codes):   # group G = pairs G, G + NG, ... (strided)
+    k = O_decode_keys_orig(key_cb_h, codes)
+    ng, ppg = key_cb_h.shape[0], key_cb_h.shape[3]
+    return k.reshape(-1, ng, ppg, 2).transpose(0, 2, 1, 3).reshape(-1, 128)
+
+
+def _bad_value_bins(w, val_codes_bh, n_codes=256):  # ignores every round after the first
+    b = O_value_bins_orig(w, val_codes_bh, n_codes)
+    b[:, 1:] = 0.0
+    return b
+
+
 O_apply_rope_orig = O.apply_rope
+O_value_bins_orig = O.value_bins
 O_decode_keys_orig = O.decode_keys
 O_decode_values_orig = O.decode_values
 
 
 @pytest.mark.parametrize("attr,bad", [("apply_rope", _bad_rope_sign), ("rope_theta", _bad_theta),
                                       ("apply_rope", _bad_pairs), ("decode_keys", _bad_decode_keys),
-                                      ("decode_values", _bad_decode_values)])
+                                      ("decode_values", _bad_decode_values),
+                                      ("decode_keys", _bad_decode_keys_strided),
+                                      ("value_bins", _bad_value_bins)])
 def test_planted_mistake_is_caught(monkeypatch, attr, bad):
     monkeypatch.setattr(O, attr, bad)
     assert not _pins_pass()

@@ -4,13 +4,14 @@ This module holds no arithmetic of the method: it only draws random tensors in t
 layouts the library and the oracle both take, so that the two sides can be compared
 on identical inputs.  Both the tests and the benchmark use it.
 
-Layouts:
+Layouts (8-scalar groups; the 64-scalar-group workloads in brackets):
   q          [B, Hq, 128]            float32 values (bf16 workloads: the exact
                                       float32 value of each bf16, plus the raw bits)
   key_cb     [Hkv, 16, R, 256, 4, 2]  float32 (re, im) of each complex codeword
-  val_cb     [Hkv, 16, R, 256, 8]     float32
-  key_codes  [B, Hkv, T_cap, R, 16]   uint8
-  val_codes  [B, Hkv, T_cap, R, 16]   uint8
+                                     [Hkv, 2, R, 64, 32, 2]
+  val_cb     [Hkv, 16, R, 256, 8]     float32  [Hkv, 2, R, 64, 64]
+  key_codes  [B, Hkv, T_cap, R, 16]   uint8    [B, Hkv, 2, R, T_cap] (planar)
+  val_codes  [B, Hkv, T_cap, R, 16]   uint8    [B, Hkv, 2, R, T_cap]
   seq_lens   [B]                      int32
   new keys / values [B, Hkv, 128]     float32 (new_tokens: one decode step's append)
 
@@ -43,6 +44,15 @@ class Workload:
     layers: int = 1
     rope_base: float = ROPE_BASE
     seed: int = 0
+    group_dim: int = 8           # scalars per quantization group: 8 or 64
+
+    @property
+    def n_groups(self) -> int:
+        return 128 // self.group_dim
+
+    @property
+    def n_codes(self) -> int:
+        return N_CODES if self.group_dim == 8 else 64
 
     @property
     def group(self) -> int:
@@ -62,6 +72,13 @@ WORKLOADS = {
                  codes="zipf1.1", lens="uniform1024-8192"),
         Workload("llama8b_32layers_B4_T65536_R2", 4, 32, 8, 65536, 2, "bf16", math.sqrt(0.5),
                  layers=32),
+        # the paper's own parameterization: 64-entry codebooks over groups of 64 scalars
+        # (32 RoPE pairs), R = 11 ("1-bit", 1.03 bits) and R = 21 ("2-bit", 1.97 bits);
+        # codebook std sqrt(1/R) so a key or value has unit variance per scalar
+        Workload("llama8b_layer_T131072_R11_g64", 1, 32, 8, 131072, 11, "f32",
+                 math.sqrt(1.0 / 11), group_dim=64),
+        Workload("llama8b_layer_T32768_R21_g64", 1, 32, 8, 32768, 21, "bf16",
+                 math.sqrt(1.0 / 21), group_dim=64),
     ]
 }
 WORKLOAD_ORDER = list(WORKLOADS)
@@ -87,10 +104,11 @@ def zipf_codes(rng: np.random.Generator, shape, s: float = 1.1) -> np.ndarray:
     return np.searchsorted(cdf, u, side="right").astype(np.uint8)
 
 
-def _codes(rng, shape, kind):
+def _codes(rng, shape, kind, n_codes=N_CODES):
     if kind == "uniform":
         n = int(np.prod(shape))
-        return np.frombuffer(rng.bytes(n), dtype=np.uint8).reshape(shape).copy()
+        c = np.frombuffer(rng.bytes(n), dtype=np.uint8).reshape(shape).copy()
+        return c if n_codes == N_CODES else c % np.uint8(n_codes)   # 256 % n_codes == 0
     if kind == "zipf1.1":
         return zipf_codes(rng, shape, 1.1)
     raise ValueError(kind)
@@ -122,14 +140,18 @@ def generate(w: Workload, layer: int = 0, t_cap: int | None = None,
         q_bits, q_val = bf16_round(q32)
     else:
         q_bits, q_val = None, q32
-    key_cb = (np.random.default_rng(s_kc).standard_normal((Hkv, 16, R, N_CODES, 4, 2),
+    NG, NC, gd = w.n_groups, w.n_codes, w.group_dim
+    key_cb = (np.random.default_rng(s_kc).standard_normal((Hkv, NG, R, NC, gd // 2, 2),
                                                           dtype=np.float32)
               * np.float32(w.cb_std)).astype(np.float32)
-    val_cb = (np.random.default_rng(s_vc).standard_normal((Hkv, 16, R, N_CODES, 8),
+    val_cb = (np.random.default_rng(s_vc).standard_normal((Hkv, NG, R, NC, gd),
                                                           dtype=np.float32)
               * np.float32(w.cb_std)).astype(np.float32)
-    key_codes = _codes(np.random.default_rng(s_kcode), (B, Hkv, T, R, 16), w.codes)
-    val_codes = _codes(np.random.default_rng(s_vcode), (B, Hkv, T, R, 16), w.codes)
+    # 8-scalar groups: token-major [B, Hkv, T, R, 16]; 64-scalar groups: planar
+    # [B, Hkv, 2, R, T] (each (group, round) row of codes contiguous over tokens)
+    code_shape = (B, Hkv, T, R, NG) if gd == 8 else (B, Hkv, NG, R, T)
+    key_codes = _codes(np.random.default_rng(s_kcode), code_shape, w.codes, NC)
+    val_codes = _codes(np.random.default_rng(s_vcode), code_shape, w.codes, NC)
     if seq_lens is None:
         seq_lens = make_seq_lens(w, B)
         seq_lens = np.minimum(seq_lens, T).astype(np.int32)
@@ -137,7 +159,8 @@ def generate(w: Workload, layer: int = 0, t_cap: int | None = None,
                 key_codes=key_codes, val_codes=val_codes,
                 seq_lens=np.asarray(seq_lens, dtype=np.int32),
                 n_q_heads=Hq, n_kv_heads=Hkv, R=R, t_cap=T, batch=B,
-                rope_base=w.rope_base)
+                rope_base=w.rope_base, group_dim=gd,
+                codes_layout="token" if gd == 8 else "planar")
 
 
 def new_tokens(w: Workload, layer: int = 0, batch: int | None = None):
@@ -152,10 +175,10 @@ def new_tokens(w: Workload, layer: int = 0, batch: int | None = None):
 
 
 def small(batch=1, n_q_heads=4, n_kv_heads=1, t_cap=64, R=1, q_dtype="f32", cb_std=1.0,
-          codes="uniform", seq_lens=None, seed=0, rope_base=ROPE_BASE) -> dict:
+          codes="uniform", seq_lens=None, seed=0, rope_base=ROPE_BASE, group_dim=8) -> dict:
     """A small custom case with the same generators (for parity and edge-case tests)."""
     w = Workload("custom", batch, n_q_heads, n_kv_heads, t_cap, R, q_dtype, cb_std,
-                 codes=codes, seed=seed, rope_base=rope_base)
+                 codes=codes, seed=seed, rope_base=rope_base, group_dim=group_dim)
     if seq_lens is None:
         seq_lens = np.full(batch, t_cap, dtype=np.int32)
     return generate(w, seq_lens=np.asarray(seq_lens, dtype=np.int32))
