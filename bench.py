@@ -264,7 +264,7 @@ def run_gpu(args):
             sets[-1].update(new_k=torch.from_numpy(nk).to(dev), new_v=torch.from_numpy(nv).to(dev),
                             pos=(sets[-1]["seq_lens"] - 1).contiguous(), host_new=(nk, nv))
     total_tokens = int(sets[0]["host"]["seq_lens"].sum())
-    shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base)
+    shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base, w.group_dim)
     if args.splits:
         S = args.splits
     elif args.form == "naive":

@@ -23,7 +23,7 @@ from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa
 
 __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
            "attend", "naive_dequant", "naive_decode", "encode_append", "split_tokens",
-           "suggest_splits", "partials_alloc", "CvqError"]
+           "suggest_splits", "partials_alloc", "group_dim_of", "CvqError"]
 
 
 def _ptr(t):
@@ -65,11 +65,21 @@ def _head_stride(cb, kind):
     raise ValueError(f"{kind} codebook has {cb.dim()} dims")
 
 
-def shape_of(q, key_codes, rope_base=500000.0):
-    """cvq_shape from q [B, Hq, 128] and key_codes [B, Hkv, T_cap, R, 16]."""
+def group_dim_of(key_cb):
+    """Scalars per quantization group, read off a key codebook [(Hkv,) NG, R, NC, PPG, 2]:
+    8 (PPG = 4, 256 codewords) or 64 (PPG = 32, 64 codewords)."""
+    return 2 * int(key_cb.shape[-2])
+
+
+def shape_of(q, key_codes, rope_base=500000.0, group_dim=8):
+    """cvq_shape from q [B, Hq, 128] and key_codes: [B, Hkv, T_cap, R, 16] (group_dim 8)
+    or planar [B, Hkv, 2, R, T_cap] (group_dim 64)."""
     B, Hq, D = q.shape
-    _, Hkv, T, R, _ = key_codes.shape
-    return make_shape(B, Hq, Hkv, R, T, rope_base, D)
+    if group_dim == 64:
+        _, Hkv, _, R, T = key_codes.shape
+    else:
+        _, Hkv, T, R, _ = key_codes.shape
+    return make_shape(B, Hq, Hkv, R, T, rope_base, D, group_dim)
 
 
 def split_tokens(shape, n_splits):
@@ -211,7 +221,7 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0
     form="table": cvq_qtable + cvq_decode_attn + cvq_combine
     form="naive": cvq_naive_dequant + cvq_naive_decode + cvq_combine (the comparison path)
     """
-    shape = shape_of(q, key_codes, rope_base)
+    shape = shape_of(q, key_codes, rope_base, group_dim_of(key_cb))
     if n_splits is None:
         n_splits = suggest_splits(shape)
     if form == "table":

@@ -29,7 +29,8 @@ class CvqError(RuntimeError):
 class cvq_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("R", ctypes.c_int32), ("t_cap", ctypes.c_int32), ("rope_base", ctypes.c_float)]
+                ("R", ctypes.c_int32), ("t_cap", ctypes.c_int32), ("rope_base", ctypes.c_float),
+                ("group_dim", ctypes.c_int32)]
 
 
 def _load():
@@ -91,5 +92,6 @@ def check(st: int, what: str):
         raise CvqError(st, f"{what}: {status_str(st)}")
 
 
-def make_shape(batch, n_q_heads, n_kv_heads, R, t_cap, rope_base=500000.0, head_dim=128):
-    return cvq_shape(batch, n_q_heads, n_kv_heads, head_dim, R, t_cap, rope_base)
+def make_shape(batch, n_q_heads, n_kv_heads, R, t_cap, rope_base=500000.0, head_dim=128,
+               group_dim=8):
+    return cvq_shape(batch, n_q_heads, n_kv_heads, head_dim, R, t_cap, rope_base, group_dim)

@@ -13,13 +13,29 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t key_cb_floats(int R) { return static_cast<size_t>(kGroups) * R * kCodes * kCodeword; }
-size_t val_cb_floats(int R) { return static_cast<size_t>(kGroups) * R * kCodes * kVDims; }
+bool is_wide(const cvq_shape* s) { return s->group_dim == kWideGroupDim; }
+
+// floats of one KV head's key / value codebook
+size_t key_cb_floats(const cvq_shape* s) {
+  return is_wide(s) ? static_cast<size_t>(kWideGroups) * s->R * kWideCodes * 2 * kWidePairs
+                    : static_cast<size_t>(kGroups) * s->R * kCodes * kCodeword;
+}
+size_t val_cb_floats(const cvq_shape* s) {
+  return is_wide(s) ? static_cast<size_t>(kWideGroups) * s->R * kWideCodes * kWideVDims
+                    : static_cast<size_t>(kGroups) * s->R * kCodes * kVDims;
+}
 
 cvq_status check_shape(const cvq_shape* s) {
   if (s == nullptr) return CVQ_ERR_NULL;
   if (s->head_dim != kHeadDim) return CVQ_ERR_UNSUPPORTED;
-  if (s->R != 1 && s->R != 2) return CVQ_ERR_UNSUPPORTED;
+  if (s->group_dim != 0 && s->group_dim != 8 && s->group_dim != kWideGroupDim)
+    return CVQ_ERR_UNSUPPORTED;
+  if (is_wide(s)) {
+    if (s->R < 1 || s->R > kWideMaxR) return CVQ_ERR_UNSUPPORTED;
+    if (s->t_cap % 16 != 0) return CVQ_ERR_SHAPE;      // planar code rows in 16-byte chunks
+  } else if (s->R != 1 && s->R != 2) {
+    return CVQ_ERR_UNSUPPORTED;
+  }
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->t_cap < 0) return CVQ_ERR_SHAPE;
   if (s->n_q_heads % s->n_kv_heads != 0) return CVQ_ERR_SHAPE;
   if (s->batch > 65535 || s->n_q_heads > 65535) return CVQ_ERR_SHAPE;
@@ -58,7 +74,7 @@ cvq_status check_decode_common(const cvq_shape* s, const uint8_t* key_codes, con
   if (seq_lens == nullptr) return CVQ_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0) return CVQ_ERR_ALIGN;
   CVQ_TRY(check_ptr(val_cb));
-  CVQ_TRY(check_stride(val_stride, val_cb_floats(s->R)));
+  CVQ_TRY(check_stride(val_stride, val_cb_floats(s)));
   if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
   CVQ_TRY(check_ptr(part_o));
   if (part_m == nullptr || part_l == nullptr) return CVQ_ERR_NULL;
@@ -130,8 +146,8 @@ const char* cvq_status_str(int status) {
 int cvq_abi_version(void) { return CVQ_ABI_VERSION; }
 
 size_t cvq_ptable_bytes(const cvq_shape* s) {
-  if (check_shape(s) != CVQ_OK) return 0;
-  return static_cast<size_t>(s->batch) * s->n_q_heads * key_cb_floats(s->R) * sizeof(float);
+  if (check_shape(s) != CVQ_OK || is_wide(s)) return 0;
+  return static_cast<size_t>(s->batch) * s->n_q_heads * key_cb_floats(s) * sizeof(float);
 }
 
 size_t cvq_partials_bytes(const cvq_shape* s, int n_splits) {
@@ -152,9 +168,12 @@ int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
   // plain kernel runs one CTA per (sequence, KV head, split).  Take the fewest splits
   // (longest, so the per-CTA codebook load and epilogue are amortized) whose CTAs fill
   // at least 90% of their last wave.
+  // With 64-scalar groups the kernel runs a cluster of 2 * ceil(R / 11) CTAs, one per SM.
   const bool clustered = (s->n_q_heads / s->n_kv_heads) == 4;
-  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads * (clustered ? 2 : 1);
-  const long long slots = static_cast<long long>(sm_count) * (clustered && s->R == 1 ? 2 : 1);
+  const long long per_split = is_wide(s) ? wide_cluster_size(s->R) : (clustered ? 2 : 1);
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads * per_split;
+  const long long slots =
+      static_cast<long long>(sm_count) * (clustered && !is_wide(s) && s->R == 1 ? 2 : 1);
   // the clustered kernel amortizes a 64R KiB codebook load per CTA, so its splits stay
   // >= 256 tokens; the plain kernel's splits may be as short as one 64-token block
   const long long min_len = clustered ? 256LL : 64LL;
@@ -170,11 +189,12 @@ int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
 cvq_status cvq_qtable(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
                       int64_t key_cb_head_stride, float* ptable, void* stream) {
   CVQ_TRY(check_shape(s));
+  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(q));
   CVQ_TRY(check_ptr(key_cb));
   CVQ_TRY(check_ptr(ptable));
-  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
   return from_cuda(launch_qtable(*s, q, q_dtype, key_cb, key_cb_head_stride, ptable,
                                  static_cast<cudaStream_t>(stream)));
 }
@@ -184,6 +204,7 @@ cvq_status cvq_decode_attn(const cvq_shape* s, const float* ptable, const uint8_
                            int64_t val_cb_head_stride, int n_splits, float* part_o, float* part_m,
                            float* part_l, void* stream) {
   CVQ_TRY(check_shape(s));
+  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(ptable));
   CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
                               n_splits, part_o, part_m, part_l));
@@ -192,7 +213,7 @@ cvq_status cvq_decode_attn(const cvq_shape* s, const float* ptable, const uint8_
   fill_common(a, s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride, n_splits, part_o,
               part_m, part_l);
   a.key_tab = ptable;
-  a.key_tab_stride = static_cast<long long>(key_cb_floats(s->R));
+  a.key_tab_stride = static_cast<long long>(key_cb_floats(s));
   return from_cuda(launch_decode_table(*s, a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -205,8 +226,10 @@ cvq_status cvq_decode_attn_gqa(const cvq_shape* s, const void* q, int q_dtype, c
   if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(q));
   CVQ_TRY(check_ptr(key_cb));
-  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
-  if ((s->n_q_heads / s->n_kv_heads) * s->R > 8) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
+  if (is_wide(s) ? (s->n_q_heads / s->n_kv_heads) != 4
+                 : (s->n_q_heads / s->n_kv_heads) * s->R > 8)
+    return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
                               n_splits, part_o, part_m, part_l));
   DecodeArgs a;
@@ -217,6 +240,7 @@ cvq_status cvq_decode_attn_gqa(const cvq_shape* s, const void* q, int q_dtype, c
   a.key_tab_stride = key_cb_head_stride;
   a.q = q;
   a.q_dtype = q_dtype;
+  if (is_wide(s)) return from_cuda(launch_decode_wide(*s, a, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -244,6 +268,7 @@ cvq_status cvq_naive_dequant(const cvq_shape* s, const float* key_cb, int64_t ke
                              const int32_t* seq_lens, const float* val_cb,
                              int64_t val_cb_head_stride, void* k_out, void* v_out, void* stream) {
   CVQ_TRY(check_shape(s));
+  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(key_cb));
   CVQ_TRY(check_ptr(val_cb));
   CVQ_TRY(check_ptr(key_codes));
@@ -252,8 +277,8 @@ cvq_status cvq_naive_dequant(const cvq_shape* s, const float* key_cb, int64_t ke
   CVQ_TRY(check_ptr(v_out));
   if (seq_lens == nullptr) return CVQ_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0) return CVQ_ERR_ALIGN;
-  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
-  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s->R)));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
+  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s)));
   PhaseTurns ph;
   phase_turns_host(s->rope_base, &ph);
   return from_cuda(launch_naive_dequant(*s, key_cb, key_cb_head_stride, val_cb, val_cb_head_stride,
@@ -287,6 +312,7 @@ cvq_status cvq_encode_append(const cvq_shape* s, const float* keys, const float*
                              int64_t val_cb_head_stride, const int32_t* positions,
                              uint8_t* key_codes, uint8_t* val_codes, void* stream) {
   CVQ_TRY(check_shape(s));
+  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(keys));
   CVQ_TRY(check_ptr(values));
   CVQ_TRY(check_ptr(key_cb));
@@ -295,8 +321,8 @@ cvq_status cvq_encode_append(const cvq_shape* s, const float* keys, const float*
   CVQ_TRY(check_ptr(val_codes));
   if (positions == nullptr) return CVQ_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(positions) & 3u) != 0) return CVQ_ERR_ALIGN;
-  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s->R)));
-  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s->R)));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
+  CVQ_TRY(check_stride(val_cb_head_stride, val_cb_floats(s)));
   if (s->t_cap == 0) return CVQ_OK;
   return from_cuda(launch_encode_append(*s, keys, values, key_cb, key_cb_head_stride, val_cb,
                                         val_cb_head_stride, positions, key_codes, val_codes,

@@ -17,6 +17,19 @@ constexpr int kVDims = 8;
 constexpr int kCodes = 256;
 constexpr int kCodeword = 8;              // floats per key codeword (4 pairs x re/im)
 constexpr int kSplitAlign = 64;           // split boundaries are multiples of this
+// the paper's own parameterization: 64-entry codebooks over groups of 64 scalars
+constexpr int kWideGroupDim = 64;
+constexpr int kWideGroups = 2;            // groups per head
+constexpr int kWidePairs = 32;            // RoPE pairs per key group
+constexpr int kWideVDims = 64;            // dims per value group
+constexpr int kWideCodes = 64;            // codewords per (group, round)
+constexpr int kWideRoundsPerCta = 11;     // rounds one CTA of the cluster holds
+constexpr int kWideMaxR = 2 * kWideRoundsPerCta;
+// CTAs per (sequence, KV head, split): one per group and round slice of <= 11 rounds
+__host__ __device__ constexpr int wide_round_slices(int R) {
+  return (R + kWideRoundsPerCta - 1) / kWideRoundsPerCta;
+}
+__host__ __device__ constexpr int wide_cluster_size(int R) { return kWideGroups * wide_round_slices(R); }
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -104,6 +117,8 @@ cudaError_t launch_naive_decode(const cvq_shape& s, const void* q, int q_dtype, 
                                 const void* v, const int32_t* seq_lens, int n_splits,
                                 int split_tokens, float* part_o, float* part_m, float* part_l,
                                 cudaStream_t stream);
+// 64-scalar groups, 4 query heads per KV head (decode_wide.cu)
+cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
 // the write side: greedy residual encoding of one new key / value per (sequence, KV head)
 cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const float* values,
                                  const float* key_cb, long long key_stride, const float* val_cb,

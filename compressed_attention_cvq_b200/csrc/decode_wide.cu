@@ -1,0 +1,363 @@
+// Split-T flash-decode over the code stream with the paper's own parameterization:
+// 64-entry codebooks over groups of 64 scalars (32 RoPE pairs share one index per round),
+// R rounds (R = 11 gives 1.03 bits per scalar, R = 21 gives 1.97), 4 query heads per KV
+// head (CommVQ summary page, "Key results" and "Limitations"; review page
+// "key_machinery").
+//
+// Work unit: one (sequence b, KV head h, split s), handled by a cluster of
+// C = 2 * ceil(R / 11) CTAs.  CTA rank rho owns group G = rho % 2 and the round slice
+// rs = rho / 2, i.e. rounds [rs * RC, rs * RC + rc) with RC = ceil(R / ceil(R / 11)).
+// Its shared memory holds those rounds' key codewords (rc x 16 KiB) and their value bins.
+//
+// Per token (8 lanes, each 4 of the group's 32 pairs):
+//   1. sum the rc key codewords of the token's codes;
+//   2. rotate each pair by its RoPE phase e^{i theta_j t} (the codeword commutes with the
+//      rotation) and project on the 4 query heads: this CTA's share of the 4 scores;
+//   3. reduce the share over the token's 8 lanes.
+// Once per 256-token tile the C CTAs exchange their shares through distributed shared
+// memory and add them in rank order, so every CTA holds bit-identical scores and runs the
+// same online softmax (a reference max per head, raised only when a tile's max exceeds it
+// by more than 8 in log2 units).  Each CTA then adds the weights to the value bins of its
+// own rounds.  Epilogue: o = bins x value codewords (staged over the key-codeword region);
+// the round slices of one group add their outputs through distributed shared memory.
+//
+// Layouts in shared memory (32 banks x 4 bytes):
+//   key / value codewords: [rc][64 codes][16 chunks of 16 bytes]; lane k of a token reads
+//     chunks k and 8 + k, so the 8 lanes of a quarter-warp read 128 contiguous bytes;
+//   bins: float r * kBinRow + c * 4 + head (kBinRow = 260, so consecutive rounds start 4
+//     banks apart);
+//   codes: [buffer][key | value][rc][256 tokens] bytes, copied with cp.async from the
+//     planar global layout [B, Hkv, 2, R, t_cap] while the previous tile computes.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace cvq {
+
+namespace {
+
+constexpr int kWHeads = 4;
+constexpr int kWTile = 256;
+constexpr int kWThreads = 512;
+constexpr int kWWarps = kWThreads / 32;
+constexpr int kWSlots = kWWarps * 4;              // tokens per step
+constexpr int kWSteps = kWTile / kWSlots;         // steps per tile
+constexpr int kWChunks = kWidePairs * 2 / 4;      // 16-byte chunks per codeword (16)
+constexpr int kBinRow = kWideCodes * kWHeads + 4; // floats per round of bins (padded)
+constexpr float kWSlack = 8.0f;
+constexpr int kRC = kWideRoundsPerCta;
+
+constexpr size_t kCwBytes = sizeof(float4) * kRC * kWideCodes * kWChunks;   // 180,224
+constexpr size_t kBinBytes = sizeof(float) * kRC * kBinRow;                 //  11,440
+constexpr size_t kXchgBytes = sizeof(float) * 2 * kWTile * kWHeads;         //   8,192
+constexpr size_t kCodeBytes = 2 * 2 * kRC * kWTile;                         //  11,264
+constexpr size_t kRedBytes = sizeof(float) * (2 * kWWarps * kWHeads + 4 * kWHeads);
+constexpr size_t kWSmem = kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kRedBytes;
+static_assert(kWSteps * kWSlots == kWTile, "tile must be a whole number of steps");
+static_assert(kWSmem <= 227 * 1024, "shared memory per CTA");
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+
+// Copy rc rounds x 64 codewords of one group (a contiguous run of rc * 4096 floats).
+__device__ __forceinline__ void stage_codebook(float4* dst, const float* src, int rc, int tid) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  const int n = rc * kWideCodes * kWChunks;
+  for (int i = tid; i < n; i += kWThreads) cp_async16(dst + i, s4 + i);
+}
+
+__global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeArgs a, int R) {
+  extern __shared__ float4 smem4[];
+  float4* cw_s = smem4;                                                       // codewords
+  float* bins = reinterpret_cast<float*>(smem4 + kRC * kWideCodes * kWChunks);
+  float* xchg = bins + kRC * kBinRow;                                         // [2][256][4]
+  uint8_t* code_s = reinterpret_cast<uint8_t*>(xchg + 2 * kWTile * kWHeads);  // [2][2][rc][256]
+  float* red_m = reinterpret_cast<float*>(code_s + kCodeBytes);              // [16][4]
+  float* red_l = red_m + kWWarps * kWHeads;                                   // [16][4]
+  float* mref_s = red_l + kWWarps * kWHeads;                                  // [4]
+  float* l_s = mref_s + kWHeads;                                              // [4]
+  float* fac_s = l_s + kWHeads;                                               // [4]
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rho = static_cast<int>(cluster.block_rank());
+  const int G = rho & 1, rs = rho >> 1;
+  const int n_slices = C >> 1;
+  const int RCeil = (R + n_slices - 1) / n_slices;
+  const int r0 = rs * RCeil;
+  const int rc = min(R, r0 + RCeil) - r0;
+
+  const int split = blockIdx.x / C;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tau = lane >> 3, k = lane & 7;
+  const int hq0 = h * kWHeads;
+
+  int L = a.seq_lens[b];
+  L = L < 0 ? 0 : (L > a.t_cap ? a.t_cap : L);
+  const int t_begin = split * a.split_tokens;
+  const int t_end = min(t_begin + a.split_tokens, L);
+  const size_t part_row = (static_cast<size_t>(b) * a.n_q_heads + hq0) * a.n_splits + split;
+
+  if (t_begin >= t_end) {   // every CTA of the cluster takes this branch
+    if (rs == 0) {
+      for (int i = tid; i < kWHeads * kWideVDims; i += kWThreads) {
+        const int hh = i / kWideVDims, d = i % kWideVDims;
+        a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + G * kWideVDims + d] = 0.f;
+      }
+    }
+    if (rho == 0 && tid < kWHeads) {
+      a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
+      a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
+    }
+    return;
+  }
+
+  // planar codes: row (b, h, G, r) of t_cap bytes
+  const size_t code_row0 = ((static_cast<size_t>(b) * a.n_kv_heads + h) * kWideGroups + G) * R + r0;
+  auto stage_codes = [&](int t_tile, int buf) {
+    const int n = 2 * rc * (kWTile / 16);
+    for (int i = tid; i < n; i += kWThreads) {
+      const int kind = i / (rc * (kWTile / 16));
+      const int r = (i / (kWTile / 16)) % rc;
+      const int q16 = i % (kWTile / 16);
+      const int t = t_tile + 16 * q16;
+      if (t < t_end) {
+        const uint8_t* src = (kind ? a.val_codes : a.key_codes) + (code_row0 + r) * a.t_cap + t;
+        cp_async16(code_s + ((buf * 2 + kind) * kRC + r) * kWTile + 16 * q16, src);
+      }
+    }
+  };
+
+  const float* kcb = a.key_tab + h * a.key_tab_stride +
+                     (static_cast<size_t>(G) * R + r0) * kWideCodes * 2 * kWidePairs;
+  stage_codebook(cw_s, kcb, rc, tid);
+  stage_codes(t_begin, 0);
+  cp_async_commit();
+  for (int i = tid; i < rc * kBinRow; i += kWThreads) bins[i] = 0.f;
+  if (tid < kWHeads) {
+    mref_s[tid] = -INFINITY;
+    l_s[tid] = 0.f;
+  }
+  for (int i = tid; i < kWWarps * kWHeads; i += kWThreads) red_l[i] = 0.f;
+
+  // this lane's 4 pairs: local pairs 2k, 2k+1 (chunk k) and 2k+16, 2k+17 (chunk 8+k)
+  int jp[4];
+  jp[0] = G * kWidePairs + 2 * k;
+  jp[1] = jp[0] + 1;
+  jp[2] = jp[0] + 16;
+  jp[3] = jp[0] + 17;
+  unsigned long long F[4];
+  float2 mul[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    F[p] = a.phase.F[jp[p]];
+    mul[p] = phase_at(F[p], kWSlots);
+  }
+  // queries, scaled to log2 units; slot j holds head (k ^ j) & 3 (select-free reduction)
+  const float qscale = kLog2e * 0.08838834764831845f;
+  float qv[kWHeads][4][2];
+#pragma unroll
+  for (int j = 0; j < kWHeads; ++j) {
+    const int hh = (k ^ j) & 3;
+    const size_t qrow = (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      qv[j][p][0] = load_q(a.q, a.q_dtype, qrow + 2 * jp[p]) * qscale;
+      qv[j][p][1] = load_q(a.q, a.q_dtype, qrow + 2 * jp[p] + 1) * qscale;
+    }
+  }
+
+  const int n_tiles = (t_end - t_begin + kWTile - 1) / kWTile;
+  const int tt0 = warp * 4 + tau;            // this lane's token slot in step 0
+  for (int it = 0; it < n_tiles; ++it) {
+    const int t_tile = t_begin + it * kWTile;
+    const int buf = it & 1;
+    cp_async_wait_all();
+    __syncthreads();                          // codes of this tile (and the codebook) landed
+    if (it + 1 < n_tiles) stage_codes(t_tile + kWTile, buf ^ 1);
+    cp_async_commit();
+    const uint8_t* kcode = code_s + (buf * 2 + 0) * kRC * kWTile;
+    const uint8_t* vcode = code_s + (buf * 2 + 1) * kRC * kWTile;
+    float* xo = xchg + buf * kWTile * kWHeads;
+
+    // ---- this CTA's share of every token's 4 scores ----
+    float2 ph[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) ph[p] = phase_at(F[p], t_tile + tt0);
+#pragma unroll 1
+    for (int step = 0; step < kWSteps; ++step) {
+      const int tt = step * kWSlots + tt0;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      if (t_tile + tt < t_end) {
+#pragma unroll
+        for (int r = 0; r < kRC; ++r) {
+          if (r < rc) {
+            const int c = kcode[r * kWTile + tt] & (kWideCodes - 1);
+            const float4* cwp = cw_s + (r * kWideCodes + c) * kWChunks;
+            const float4 x = cwp[k], y = cwp[8 + k];
+            acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
+            acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+          }
+        }
+      }
+      float P[kWHeads] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float xr = acc[2 * p], xi = acc[2 * p + 1];
+        const float zr = fmaf(ph[p].x, xr, -ph[p].y * xi);
+        const float zi = fmaf(ph[p].x, xi, ph[p].y * xr);
+#pragma unroll
+        for (int j = 0; j < kWHeads; ++j) P[j] = fmaf(qv[j][p][0], zr, fmaf(qv[j][p][1], zi, P[j]));
+      }
+      // sum over the token's 8 lanes; lane k ends with head k & 3
+      const float s0 = P[0] + __shfl_xor_sync(0xffffffffu, P[2], 2);
+      const float s1 = P[1] + __shfl_xor_sync(0xffffffffu, P[3], 2);
+      float v = s0 + __shfl_xor_sync(0xffffffffu, s1, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      if (k < kWHeads) xo[tt * kWHeads + k] = v;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) ph[p] = cmul(ph[p], mul[p]);
+    }
+
+    // ---- exchange: every CTA sums the C shares in rank order ----
+    cluster_sync_all();
+    const int hh = tid & 3;
+    const int tA = tid >> 2, tB = tA + kWTile / 2;
+    float sA = 0.f, sB = 0.f;
+    for (int q = 0; q < C; ++q) {
+      const float* px = cluster.map_shared_rank(xo, q);
+      sA += px[tA * kWHeads + hh];
+      sB += px[tB * kWHeads + hh];
+    }
+    if (t_tile + tA >= t_end) sA = -INFINITY;
+    if (t_tile + tB >= t_end) sB = -INFINITY;
+
+    // ---- online softmax with a lagging reference max ----
+    float mx = fmaxf(sA, sB);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (lane < kWHeads) red_m[warp * kWHeads + lane] = mx;
+    __syncthreads();
+    if (tid < kWHeads) {
+      float tm = -INFINITY, pend = 0.f;
+      for (int w = 0; w < kWWarps; ++w) {
+        tm = fmaxf(tm, red_m[w * kWHeads + tid]);
+        pend += red_l[w * kWHeads + tid];    // the previous tile's weights
+      }
+      const float mo = mref_s[tid];
+      float f = 1.f;
+      if (tm > mo + kWSlack) {
+        f = (mo == -INFINITY) ? 0.f : exp2f(mo - tm);
+        mref_s[tid] = tm;
+      }
+      l_s[tid] = (l_s[tid] + pend) * f;
+      fac_s[tid] = f;
+    }
+    __syncthreads();
+    if (fac_s[0] != 1.f || fac_s[1] != 1.f || fac_s[2] != 1.f || fac_s[3] != 1.f) {
+      for (int i = tid; i < rc * kBinRow; i += kWThreads) bins[i] *= fac_s[i & 3];
+      __syncthreads();
+    }
+    const float m = mref_s[hh];
+    const float wA = exp2f(sA - m), wB = exp2f(sB - m);
+    float ls = wA + wB;
+    ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+    ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+    ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+    if (lane < kWHeads) red_l[warp * kWHeads + lane] = ls;
+    // value reorder: the weight goes to the bin of the token's value code, per own round
+    if (wA > 0.f) {
+      for (int r = 0; r < rc; ++r)
+        atomicAdd(&bins[r * kBinRow + (vcode[r * kWTile + tA] & (kWideCodes - 1)) * kWHeads + hh], wA);
+    }
+    if (wB > 0.f) {
+      for (int r = 0; r < rc; ++r)
+        atomicAdd(&bins[r * kBinRow + (vcode[r * kWTile + tB] & (kWideCodes - 1)) * kWHeads + hh], wB);
+    }
+  }
+  __syncthreads();
+  if (tid < kWHeads) {
+    float pend = 0.f;
+    for (int w = 0; w < kWWarps; ++w) pend += red_l[w * kWHeads + tid];
+    l_s[tid] += pend;
+  }
+
+  // ---- epilogue: o = bins x value codewords of the own rounds ----
+  const float* vcb = a.val_cb + h * a.val_cb_stride +
+                     (static_cast<size_t>(G) * R + r0) * kWideCodes * kWideVDims;
+  stage_codebook(cw_s, vcb, rc, tid);
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  const float* cv = reinterpret_cast<const float*>(cw_s);
+  const int eh = (tid >> 6) & 3, ed = tid & 63, half = tid >> 8;
+  float o = 0.f;
+  for (int r = 0; r < rc; ++r) {
+    const float* br = bins + r * kBinRow + eh;
+    const float* vr = cv + static_cast<size_t>(r) * kWideCodes * kWideVDims + ed;
+#pragma unroll 8
+    for (int c = half * 32; c < half * 32 + 32; ++c) o = fmaf(br[c * kWHeads], vr[c * kWideVDims], o);
+  }
+  // the xchg buffer the last tile did not use: no peer reads it any more
+  float* ored = xchg + (n_tiles & 1) * kWTile * kWHeads;   // [256] halves, then [256] slice
+  float* oslice = ored + kWHeads * kWideVDims;
+  if (half) ored[eh * kWideVDims + ed] = o;
+  __syncthreads();
+  if (!half) {
+    o += ored[eh * kWideVDims + ed];
+    if (rs == 1) oslice[eh * kWideVDims + ed] = o;
+  }
+  cluster_sync_all();          // slices written; peers are done reading this CTA's xchg
+  if (!half && rs == 0) {
+    if (n_slices == 2) o += cluster.map_shared_rank(oslice, rho + 2)[eh * kWideVDims + ed];
+    a.part_o[(part_row + static_cast<size_t>(eh) * a.n_splits) * kHeadDim + G * kWideVDims + ed] = o;
+  }
+  if (rho == 0 && tid < kWHeads) {
+    a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = mref_s[tid] * kLn2;
+    a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = l_s[tid];
+  }
+  cluster_sync_all();          // keep oslice alive until the peer has read it
+}
+
+}  // namespace
+
+cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
+  const int C = wide_cluster_size(s.R);
+  cudaError_t e = cudaFuncSetAttribute(decode_wide_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kWSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_splits * C), s.n_kv_heads, s.batch);
+  cfg.blockDim = dim3(kWThreads);
+  cfg.dynamicSmemBytes = kWSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_wide_kernel, a, s.R);
+}
+
+}  // namespace cvq

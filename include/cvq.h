@@ -11,13 +11,23 @@
  * accumulated per value code before the value codebook multiply (review page,
  * "forward_implications", 4th item).
  *
- * The instance implemented here:
- *   head_dim 128 = 64 interleaved RoPE pairs (2j, 2j+1), theta_j = base^(-2j/128);
- *   key:   16 groups of 4 pairs, R rounds, 256 complex codewords per (group, round);
- *   value: 16 groups of 8 dims,  R rounds, 256 codewords per (group, round);
+ * Two instances (cvq_shape.group_dim), both with head_dim 128 = 64 interleaved RoPE
+ * pairs (2j, 2j+1), theta_j = base^(-2j/128), and a group of g consecutive scalars
+ * sharing one index per round (review page, "key_machinery"):
+ *   g = 8  (default): key 16 groups of 4 pairs, value 16 groups of 8 dims, 256
+ *          codewords per (group, round), R = 1 or 2 -> 1 or 2 bits per scalar;
+ *          codes token-major [B, Hkv, t_cap, R, 16];
+ *   g = 64 (the paper's own parameterization; CommVQ summary page, "Key results" and
+ *          "Limitations"): key 2 groups of 32 pairs, value 2 groups of 64 dims, 64
+ *          codewords per (group, round), R = 1..22 (11 -> 1.03 bits, 21 -> 1.97 bits
+ *          per scalar; each 6-bit code is stored in one uint8);
+ *          codes planar [B, Hkv, 2, R, t_cap], t_cap a multiple of 16.
  *   score_t = sum_j Re(e^{i theta_j t} conj(q_j) sum_r c_{t,r,j}) / sqrt(128), t = 0..L-1
  *   out = sum_t softmax(score)_t v_t,   lse = ln sum_t exp(score_t).
  * Query head hq reads KV head hq / (n_q_heads / n_kv_heads).
+ * Every entry point takes g = 8; cvq_decode_attn_gqa (4 query heads per KV head),
+ * cvq_attend_static, cvq_combine and the size helpers also take g = 64; the others
+ * return CVQ_ERR_UNSUPPORTED for it.
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers, owned by the caller, row-major, and
@@ -45,7 +55,7 @@ extern "C" {
 #define CVQ_API
 #endif
 
-#define CVQ_ABI_VERSION 1
+#define CVQ_ABI_VERSION 2
 #define CVQ_HEAD_DIM 128
 #define CVQ_GROUPS 16
 #define CVQ_CODES 256
@@ -68,9 +78,10 @@ typedef struct {
   int32_t n_q_heads;  /* Hq >= 1, a multiple of n_kv_heads                   */
   int32_t n_kv_heads; /* Hkv >= 1; Hq/Hkv in {1, 2, 4, 8}                     */
   int32_t head_dim;   /* must be 128                                          */
-  int32_t R;          /* residual rounds, 1 or 2                              */
+  int32_t R;          /* residual rounds: 1 or 2 (g = 8), 1..22 (g = 64)      */
   int32_t t_cap;      /* token capacity of the code buffers per sequence, >= 0 */
   float rope_base;    /* RoPE base, > 1 (500000 for LLaMA-3.1)                */
+  int32_t group_dim;  /* scalars per quantization group: 0 or 8 (default), 64 */
 } cvq_shape;
 
 /* Human-readable name of a status code (static storage). */
@@ -148,6 +159,13 @@ CVQ_API cvq_status cvq_decode_attn(const cvq_shape* shape, const float* ptable, 
  *     Re(e^{i theta t} conj(q) c) = Re(conj(q) (e^{i theta t} c)).
  *   q, q_dtype, key_cb, key_cb_head_stride as in cvq_qtable; the rest as in
  *   cvq_decode_attn.
+ *   With group_dim = 64 (Hq / Hkv must be 4):
+ *     key_cb     [Hkv][2, R, 64, 32, 2] fp32 (group G, round r, code c, pair p, re/im;
+ *                pair j = 32 G + p), stride 0 or >= 2*R*64*64 floats
+ *     val_cb     [Hkv][2, R, 64, 64] fp32 (value dim 64 G + d), same stride rule
+ *     key_codes, val_codes  planar [B, Hkv, 2, R, t_cap] uint8 (the low 6 bits of
+ *                each byte are the code; the top 2 bits are ignored), t_cap a multiple
+ *                of 16 (else CVQ_ERR_SHAPE)
  * ------------------------------------------------------------------------------- */
 CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, int q_dtype,
                                const float* key_cb, int64_t key_cb_head_stride,

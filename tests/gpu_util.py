@@ -33,7 +33,8 @@ def run_gpu(d, form="gqa", n_splits=None, dd=None):
 
 def run_oracle(d, heads=None):
     return O.attend(d["q"], d["key_cb"], d["val_cb"], d["key_codes"], d["val_codes"],
-                    d["seq_lens"], d["rope_base"], heads=heads)
+                    d["seq_lens"], d["rope_base"], heads=heads,
+                    codes_layout=d.get("codes_layout", "token"))
 
 
 def assert_close(out, lse, ref_out, ref_lse, heads=None, out_tol=OUT_TOL, lse_rtol=LSE_RTOL):

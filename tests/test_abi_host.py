@@ -26,8 +26,9 @@ def _shape(**kw):
     d = dict(batch=1, n_q_heads=32, n_kv_heads=8, R=2, t_cap=1024, rope_base=500000.0)
     d.update(kw)
     head_dim = d.pop("head_dim", 128)
+    group_dim = d.pop("group_dim", 8)
     return b.make_shape(d["batch"], d["n_q_heads"], d["n_kv_heads"], d["R"], d["t_cap"],
-                        d["rope_base"], head_dim)
+                        d["rope_base"], head_dim, group_dim)
 
 
 def test_every_declared_symbol_is_exported():
@@ -182,3 +183,25 @@ def test_encode_append_errors():
     assert _encode(s, kstride=65536 + 1) == 3
     assert _encode(_shape(R=3)) == 4
     assert _encode(_shape(t_cap=0)) == 0           # nothing to write, no launch
+
+
+def test_wide_layout_validation():
+    """group_dim 64 (64-entry codebooks over 64-scalar groups): R up to 22, t_cap a
+    multiple of 16, 4 query heads per KV head; only the GQA decode, the static entry,
+    combine and the size helpers take it."""
+    w = dict(group_dim=64, R=11, t_cap=1024)
+    assert _gqa(_shape(**w), kcb=None) == 1                          # R = 11 accepted
+    assert _gqa(_shape(**dict(w, R=23))) == 4
+    assert _gqa(_shape(**dict(w, R=0))) == 4
+    assert _gqa(_shape(**dict(w, t_cap=1000))) == 2                  # not a multiple of 16
+    assert _gqa(_shape(**dict(w, n_q_heads=16))) == 4                # 2 heads per KV head
+    assert _gqa(_shape(**w), kstride=8192 * 11 - 4) == 2             # below one head
+    assert _gqa(_shape(**w), kstride=8192 * 11 + 2) == 3
+    assert _gqa(_shape(group_dim=32)) == 4
+    assert _qtable(_shape(**w)) == 4
+    assert _decode(_shape(**w)) == 4
+    assert _encode(_shape(**w)) == 4
+    assert b.lib.cvq_ptable_bytes(ctypes.byref(_shape(**w))) == 0
+    assert b.lib.cvq_partials_bytes(ctypes.byref(_shape(**w)), 3) == 32 * 3 * 130 * 4
+    assert b.lib.cvq_suggest_splits(ctypes.byref(_shape(**dict(w, t_cap=131072))), 148) == 9
+    assert b.lib.cvq_suggest_splits(ctypes.byref(_shape(**dict(w, t_cap=32768, R=21))), 148) == 9
