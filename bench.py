@@ -48,17 +48,19 @@ N_INPUT_SETS = 8
 
 def algorithmic_flops(w: workloads.Workload, total_tokens: int) -> float:
     """Algorithmic FP32 work of one layer step (per token per query head: 64 pairs x
-    (2 mul + 2 add) = 256, plus 128 (R - 1) adds to sum the rounds, plus 16 R bin adds;
-    exp and sin/cos are counted on the SFU, not here)."""
-    per_tok_head = 256 + 128 * (w.R - 1) + 16 * w.R
+    (2 mul + 2 add) = 256, plus 128 (R - 1) adds to sum the rounds, plus one bin add per
+    (group, round): 16 R, or 2 R with 64-scalar groups; exp and sin/cos are counted on
+    the SFU, not here)."""
+    per_tok_head = 256 + 128 * (w.R - 1) + w.n_groups * w.R
     return float(total_tokens) * w.n_q_heads * per_tok_head
 
 
 def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
     """Bytes that must come from HBM per layer step: key + value codes of every token of
-    every KV head, plus the key and value codebooks of every KV head."""
-    codes = float(total_tokens) * w.n_kv_heads * 32 * w.R
-    cbs = 2.0 * w.n_kv_heads * 16 * w.R * 256 * 8 * 4
+    every KV head (one byte per group and round), plus the key and value codebooks of
+    every KV head."""
+    codes = float(total_tokens) * w.n_kv_heads * 2 * w.n_groups * w.R
+    cbs = 2.0 * w.n_kv_heads * w.n_groups * w.R * w.n_codes * w.group_dim * 4
     return codes + cbs
 
 
@@ -197,6 +199,8 @@ def oracle_sample(w: workloads.Workload, budget_s: float = 12.0, layer: int = 0)
     from oracle import cvq_oracle as O
 
     d = workloads.generate(w, layer=layer)
+    if d["codes_layout"] == "planar":
+        d["key_codes"], d["val_codes"] = O.token_major(d["key_codes"]), O.token_major(d["val_codes"])
     lens = d["seq_lens"]
     total_tokens = int(lens.sum())
     heads = [(b, h) for b in range(w.batch) for h in range(w.n_q_heads)]

@@ -20,8 +20,9 @@ definition states):
   4. score_t = q . RoPE_t(k_t) / sqrt(128), q being the already-rotated query.
   5. Softmax with max subtraction; lse = m + ln(sum exp(s - m)).
   6. Each value is reconstructed as an additive sum of R codewords per group of VD
-     dims ("decoded via simple matrix multiplication" -- CommVQ abstract, on the
-     aitopics.org "1-bit quantization" page), and out = sum_t w_t v_t.
+     dims (the CommVQ abstract on the aitopics.org "1-bit quantization" page: a value
+     is recovered from its codes by a plain matrix product with the codebook), and
+     out = sum_t w_t v_t.
 
 Also here, each following the same pages:
   * qtable(): the query x key-codebook table P = conj(q_j) * c that the method
@@ -44,8 +45,8 @@ Layouts (all row-major):
   seq_lens   [B] int
 Query head hq reads KV head hq // (Hq // Hkv).  A group G is PPG consecutive RoPE
 pairs of the key (pairs PPG*G .. PPG*G + PPG - 1) and VD = 2*PPG consecutive dims of
-the value ("consecutive sub-vectors share one quantized index (group size g)" --
-review page, "key_machinery").  Two instances are used, read off the codebook shapes:
+the value (the review page, "key_machinery": neighbouring sub-vectors use the same
+quantization index, g of them per group).  Two instances are used, read off the codebook shapes:
   g = 8 scalars:  NG = 16, PPG = 4,  NC = 256 codewords, R = 1 or 2 (1 or 2 bits);
   g = 64 scalars: NG = 2,  PPG = 32, NC = 64 codewords,  R = 11 or 21 -- the paper's own
                   parameterization, R log2(64) / 64 = 1.03 or 1.97 bits (CommVQ summary
