@@ -1,12 +1,14 @@
 """Benchmark: CommVQ decode attention, KV tokens/s per layer on B200.
 
-    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--form gqa|table|naive]
-                    [--append]
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
+                    [--form gqa|gqa_split|table|naive] [--append]
     python bench.py --impl reference ...     # the float64 CPU oracle, timed on host cores
 
 A step is one decode-attention pass over one layer of the workload: every query head
-of every sequence against its whole cached code stream (decode + combine; the table
-form adds the query-table build).  Inputs are resident in HBM before timing; 8
+of every sequence against its whole cached code stream.  The default form is one launch
+(cvq_attend: the decode with the split merge fused into its last CTA per unit);
+gqa_split runs the decode and cvq_combine as two launches, the table form adds the
+query-table build, naive decodes the cache to fp16 first.  Inputs are resident in HBM before timing; 8
 independent layer-sized input sets rotate from step to step so no step finds the
 previous one's codes in L2 (8 x 36 MB > 126 MB L2 for the 128K layer).  With --append
 the step also writes the step's new key and value of every (sequence, KV head) into the
@@ -89,7 +91,7 @@ def recorded_traffic(workload: str, form: str):
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if form != "gqa" or not os.path.exists(path):
+    if form not in ("gqa", "gqa_split") or not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
@@ -277,6 +279,7 @@ def run_gpu(args):
     else:
         S = cvq.suggest_splits(shape)
     parts = cvq.partials_alloc(shape, S, dev)
+    ws = cvq.workspace_alloc(shape, S, dev) if args.form == "gqa" else None
     out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
     ptab = (torch.empty((w.batch, w.n_q_heads, 16, w.R, 256, 4, 2), dtype=torch.float32, device=dev)
@@ -286,17 +289,23 @@ def run_gpu(args):
         kh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
         vh = torch.zeros(kv_dims, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = (3 if args.form in ("table", "naive") else 2) + (1 if args.append else 0)
+    launches_per_step = ({"gqa": 1, "gqa_split": 2}.get(args.form, 3)
+                         + (1 if args.append else 0))
+
+    # Events: one at the start of the timed region, then per step one after the append (if
+    # any), one after the decode (if a combine follows) and one at the end of the step; the
+    # end of a step is the start of the next.  Each event record costs the stream ~2.6 us, so
+    # no event is recorded where nothing runs between two of them.
+    def mark(ev, key):
+        if ev is not None:
+            ev[key].record(stream)
 
     def step(i, ev=None):
         s = sets[i % n_sets]
-        if ev is not None:
-            ev[0].record(stream)
         if args.append:
             cvq.encode_append(shape, s["new_k"], s["new_v"], s["key_cb"], s["val_cb"], s["pos"],
                               s["key_codes"], s["val_codes"])
-        if ev is not None:
-            ev[3].record(stream)
+            mark(ev, "enc")
         if args.form == "table":
             cvq.qtable(shape, s["q"], s["key_cb"], ptable=ptab)
             cvq.decode_attn(shape, ptab, s["key_codes"], s["val_codes"], s["seq_lens"], s["val_cb"],
@@ -305,19 +314,23 @@ def run_gpu(args):
             cvq.naive_dequant(shape, s["key_cb"], s["val_cb"], s["key_codes"], s["val_codes"],
                               s["seq_lens"], k_out=kh, v_out=vh)
             cvq.naive_decode(shape, s["q"], kh, vh, s["seq_lens"], S, partials=parts)
-        else:
+        elif args.form == "gqa_split":
             cvq.decode_attn_gqa(shape, s["q"], s["key_cb"], s["key_codes"], s["val_codes"],
                                 s["seq_lens"], s["val_cb"], S, partials=parts)
-        if ev is not None:
-            ev[1].record(stream)
-        cvq.combine(shape, S, *parts, out=out, lse=lse)
-        if ev is not None:
-            ev[2].record(stream)
+        else:
+            cvq.attend_fused(shape, s["q"], s["key_cb"], s["key_codes"], s["val_codes"],
+                             s["seq_lens"], s["val_cb"], S, workspace=ws, out=out, lse=lse)
+        if args.form != "gqa":
+            mark(ev, "dec")
+            cvq.combine(shape, S, *parts, out=out, lse=lse)
+        mark(ev, "end")
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    keys = (["enc"] if args.append else []) + (["dec"] if args.form != "gqa" else []) + ["end"]
+    evs = [{k: torch.cuda.Event(enable_timing=True) for k in keys} for _ in range(args.steps)]
+    ev_start = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -325,13 +338,16 @@ def run_gpu(args):
         time.sleep(0.25)   # let the sampler start
         torch.cuda.synchronize()
         for i in range(args.steps):
+            if i == 0:
+                ev_start.record(stream)
             step(args.warmup + i, evs[i])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[3].elapsed_time(e[1]) for e in evs]
-    enc_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    starts = [ev_start] + [e["end"] for e in evs[:-1]]
+    step_ms = [a.elapsed_time(e["end"]) for a, e in zip(starts, evs)]
+    dec_ms = [e.get("enc", a).elapsed_time(e.get("dec", e["end"])) for a, e in zip(starts, evs)]
+    enc_ms = [a.elapsed_time(e["enc"]) for a, e in zip(starts, evs)] if args.append else []
     total_ms_max = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms_max / args.steps
 
@@ -363,9 +379,14 @@ def run_gpu(args):
             cvq.encode_append(shape, dev_in["new_k"], dev_in["new_v"], dev_in["key_cb"],
                               dev_in["val_cb"], dev_in["pos"], dev_in["key_codes"],
                               dev_in["val_codes"])
-        o, l = cvq.attend(dev_in["q"], dev_in["key_cb"], dev_in["val_cb"], dev_in["key_codes"],
-                          dev_in["val_codes"], dev_in["seq_lens"], w.rope_base, n_splits=S,
-                          form=args.form)
+        if args.form == "gqa":
+            o, l = cvq.attend_fused(shape, dev_in["q"], dev_in["key_cb"], dev_in["key_codes"],
+                                    dev_in["val_codes"], dev_in["seq_lens"], dev_in["val_cb"], S,
+                                    workspace=ws, out=out, lse=lse)
+        else:
+            o, l = cvq.attend(dev_in["q"], dev_in["key_cb"], dev_in["val_cb"],
+                              dev_in["key_codes"], dev_in["val_codes"], dev_in["seq_lens"],
+                              w.rope_base, n_splits=S, form=args.form)
         host_out.copy_(o, non_blocking=True)
         host_lse.copy_(l, non_blocking=True)
 
@@ -472,8 +493,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
-    ap.add_argument("--form", choices=["gqa", "table", "naive"], default="gqa",
-                    help="gqa: the library's fast path; table: the pages' per-query-head table "
+    ap.add_argument("--form", choices=["gqa", "gqa_split", "table", "naive"], default="gqa",
+                    help="gqa: the library's fast path, one launch; gqa_split: decode and "
+                         "combine as two launches; table: the pages' per-query-head table "
                          "form; naive: decode the cache to fp16 then attend (comparison path)")
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--append", action="store_true",

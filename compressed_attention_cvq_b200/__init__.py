@@ -1,13 +1,16 @@
 """CommVQ decode attention on B200: Python binding of libcvq.
 
-The three calls of the library, one-to-one with include/cvq.h:
+The calls of the library, one-to-one with include/cvq.h:
 
   qtable(shape, q, key_cb)                       -> P table      (cvq_qtable)
   decode_attn(shape, ptable, codes..., n_splits) -> partials     (cvq_decode_attn)
   decode_attn_gqa(shape, q, key_cb, codes...)    -> partials     (cvq_decode_attn_gqa)
   combine(shape, partials)                       -> (out, lse)   (cvq_combine)
+  attend_fused(shape, q, key_cb, codes...)       -> (out, lse)   (cvq_attend)
+  naive_dequant / naive_decode                   -> the comparison path
+  encode_append(shape, keys, values, ...)        -> codes written (cvq_encode_append)
 
-plus attend(), which allocates the partial states with torch and runs the calls in
+plus attend(), which allocates the intermediate buffers with torch and runs the calls in
 order.  Tensors are torch CUDA tensors in the layouts documented in cvq.h; work is
 enqueued on torch's current CUDA stream.  torch provides device memory and streams
 only: every arithmetic step runs in the library's CUDA kernels.
@@ -23,7 +26,8 @@ from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa
 
 __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
            "attend", "naive_dequant", "naive_decode", "encode_append", "split_tokens",
-           "suggest_splits", "partials_alloc", "group_dim_of", "CvqError"]
+           "suggest_splits", "partials_alloc", "group_dim_of", "attend_fused", "workspace_alloc",
+           "CvqError"]
 
 
 def _ptr(t):
@@ -152,6 +156,37 @@ def decode_attn_gqa(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_
     return part_o, part_m, part_l
 
 
+def workspace_alloc(shape, n_splits, device):
+    """Zeroed workspace for attend_fused (the partial states and the arrival counters,
+    which every call leaves zero again)."""
+    n = _b.lib.cvq_attend_workspace_bytes(ctypes.byref(shape), n_splits)
+    if n == 0:
+        raise ValueError("invalid shape or n_splits for cvq_attend_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def attend_fused(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
+                 workspace=None, out=None, lse=None, stream=None):
+    """GQA decode with the split merge fused into its last CTA per work unit: one launch
+    (cvq_attend).  Returns (out [B, Hq, 128], lse [B, Hq])."""
+    _require(q, "q", (torch.float32, torch.bfloat16))
+    _require(key_cb, "key_cb", torch.float32)
+    _codes_check(key_codes, val_codes, seq_lens, val_cb)
+    dev = key_codes.device
+    if workspace is None:
+        workspace = workspace_alloc(shape, n_splits, dev)
+    if out is None:
+        out = torch.empty((shape.batch, shape.n_q_heads, 128), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((shape.batch, shape.n_q_heads), dtype=torch.float32, device=dev)
+    st = _b.lib.cvq_attend(ctypes.byref(shape), _ptr(q), _q_dtype(q), _ptr(key_cb),
+                           _head_stride(key_cb, "key"), _ptr(key_codes), _ptr(val_codes),
+                           _ptr(seq_lens), _ptr(val_cb), _head_stride(val_cb, "val"), n_splits,
+                           _ptr(workspace), _ptr(out), _ptr(lse), _stream(stream))
+    _b.check(st, "cvq_attend")
+    return out, lse
+
+
 def combine(shape, n_splits, part_o, part_m, part_l, out=None, lse=None, stream=None):
     if out is None:
         out = torch.empty((shape.batch, shape.n_q_heads, 128), dtype=torch.float32,
@@ -217,7 +252,8 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0
            form="gqa", stream=None):
     """One decode step: (out [B, Hq, 128], lse [B, Hq]) in fp32.
 
-    form="gqa":   cvq_decode_attn_gqa + cvq_combine
+    form="gqa":   cvq_attend (decode with the merge fused in: one launch)
+    form="gqa_split": cvq_decode_attn_gqa + cvq_combine
     form="table": cvq_qtable + cvq_decode_attn + cvq_combine
     form="naive": cvq_naive_dequant + cvq_naive_decode + cvq_combine (the comparison path)
     """
@@ -231,6 +267,9 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0
         kh, vh = naive_dequant(shape, key_cb, val_cb, key_codes, val_codes, seq_lens, stream=stream)
         parts = naive_decode(shape, q, kh, vh, seq_lens, n_splits, stream=stream)
     elif form == "gqa":
+        return attend_fused(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
+                            stream=stream)
+    elif form == "gqa_split":
         parts = decode_attn_gqa(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_splits,
                                 stream=stream)
     else:

@@ -103,6 +103,40 @@ void fill_common(DecodeArgs& a, const cvq_shape* s, const uint8_t* key_codes, co
   phase_turns_host(s->rope_base, &a.phase);
 }
 
+size_t round16(size_t n) { return (n + 15) / 16 * 16; }
+
+// The GQA-form decode; with counters != nullptr the last CTA of every work unit also merges
+// the split partials into out and lse (cvq_attend).
+cvq_status decode_gqa_impl(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                           int64_t key_cb_head_stride, const uint8_t* key_codes,
+                           const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                           int64_t val_cb_head_stride, int n_splits, float* part_o, float* part_m,
+                           float* part_l, int* counters, float* out, float* lse, void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_ptr(q));
+  CVQ_TRY(check_ptr(key_cb));
+  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
+  if (is_wide(s) ? (s->n_q_heads / s->n_kv_heads) != 4
+                 : (s->n_q_heads / s->n_kv_heads) * s->R > 8)
+    return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
+                              n_splits, part_o, part_m, part_l));
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fill_common(a, s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride, n_splits, part_o,
+              part_m, part_l);
+  a.key_tab = key_cb;
+  a.key_tab_stride = key_cb_head_stride;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.counters = counters;
+  a.out = out;
+  a.lse = lse;
+  if (is_wide(s)) return from_cuda(launch_decode_wide(*s, a, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace
 
 namespace cvq {
@@ -222,26 +256,38 @@ cvq_status cvq_decode_attn_gqa(const cvq_shape* s, const void* q, int q_dtype, c
                                const uint8_t* val_codes, const int32_t* seq_lens,
                                const float* val_cb, int64_t val_cb_head_stride, int n_splits,
                                float* part_o, float* part_m, float* part_l, void* stream) {
+  return decode_gqa_impl(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
+                         seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
+                         nullptr, nullptr, nullptr, stream);
+}
+
+size_t cvq_attend_workspace_bytes(const cvq_shape* s, int n_splits) {
+  const size_t parts = cvq_partials_bytes(s, n_splits);
+  if (parts == 0) return 0;
+  return round16(parts) + round16(static_cast<size_t>(s->batch) * s->n_q_heads * sizeof(int));
+}
+
+cvq_status cvq_attend(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                      int64_t key_cb_head_stride, const uint8_t* key_codes,
+                      const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                      int64_t val_cb_head_stride, int n_splits, void* workspace, float* out,
+                      float* lse, void* stream) {
   CVQ_TRY(check_shape(s));
-  if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
-  CVQ_TRY(check_ptr(q));
-  CVQ_TRY(check_ptr(key_cb));
-  CVQ_TRY(check_stride(key_cb_head_stride, key_cb_floats(s)));
-  if (is_wide(s) ? (s->n_q_heads / s->n_kv_heads) != 4
-                 : (s->n_q_heads / s->n_kv_heads) * s->R > 8)
-    return CVQ_ERR_UNSUPPORTED;
-  CVQ_TRY(check_decode_common(s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride,
-                              n_splits, part_o, part_m, part_l));
-  DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  fill_common(a, s, key_codes, val_codes, seq_lens, val_cb, val_cb_head_stride, n_splits, part_o,
-              part_m, part_l);
-  a.key_tab = key_cb;
-  a.key_tab_stride = key_cb_head_stride;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  if (is_wide(s)) return from_cuda(launch_decode_wide(*s, a, static_cast<cudaStream_t>(stream)));
-  return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
+  CVQ_TRY(check_ptr(workspace));
+  CVQ_TRY(check_ptr(out));
+  if (lse == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return CVQ_ERR_ALIGN;
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  // workspace: part_o [rows][128], part_m [rows], part_l [rows], then the counters
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_m = part_o + rows * kHeadDim;
+  float* part_l = part_m + rows;
+  int* counters = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                         round16(rows * (kHeadDim + 2) * sizeof(float)));
+  return decode_gqa_impl(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
+                         seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
+                         counters, out, lse, stream);
 }
 
 cvq_status cvq_combine(const cvq_shape* s, int n_splits, const float* part_o, const float* part_m,

@@ -98,7 +98,94 @@ struct DecodeArgs {
   float* part_m;
   float* part_l;
   PhaseTurns phase;
+  // fused merge (cvq_attend): arrival counters per work unit and the final outputs;
+  // counters == nullptr leaves the merge to cvq_combine
+  int* counters;
+  float* out;
+  float* lse;
 };
+
+// The split merge of cvq_combine, fused into the end of a decode kernel.  Every CTA of a
+// work unit (sequence b, grid row `unit` = blockIdx.y) calls this with all its threads
+// after writing its partial states; `expected` CTAs write the unit's partials.  The CTA
+// that arrives last merges the unit's n_heads query heads (hq0 ..) into out and lse with
+// the arithmetic of combine_kernel, in the same order, and clears the counter for the
+// next call.  No CTA waits for another: the others simply finish.
+__device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit, int hq0,
+                                           int n_heads, int expected) {
+  int* ctr = a.counters + static_cast<size_t>(b) * gridDim.y + unit;
+  int old = 0;
+  __syncthreads();                       // this CTA's partial states are all written
+  if (threadIdx.x == 0) {
+    __threadfence();                     // ... and visible device-wide before the count
+    old = atomicAdd(ctr, 1);
+  }
+  if (!__syncthreads_or(threadIdx.x == 0 && old == expected - 1)) return;
+  __threadfence();
+  // One warp per query head; lane l owns output dims l, l + 32, l + 64, l + 96.  Loads are
+  // issued 4 splits at a time, one group ahead of its use (they do not depend on M), and the
+  // sums run over the splits in order, as in combine_kernel.
+  constexpr int kU = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.n_splits;
+  for (int hh = warp; hh < n_heads; hh += blockDim.x >> 5) {
+    const size_t row = static_cast<size_t>(b) * a.n_q_heads + hq0 + hh;
+    const float* pm = a.part_m + row * S;
+    const float* pl = a.part_l + row * S;
+    const float* po = a.part_o + row * S * kHeadDim + lane;
+    float x[kU][4];
+    auto load_o = [&](int s0) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x[u][j] = s0 + u < S ? __ldcg(po + static_cast<size_t>(s0 + u) * kHeadDim + 32 * j) : 0.f;
+      }
+    };
+    float mv = lane < S ? __ldcg(pm + lane) : -INFINITY;    // splits 0..31
+    float lv = lane < S ? __ldcg(pl + lane) : 0.f;
+    load_o(0);
+    float M = mv;
+    for (int s = lane + 32; s < S; s += 32) M = fmaxf(M, __ldcg(pm + s));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float* orow = a.out + row * kHeadDim + lane;
+    if (M == -INFINITY) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) orow[32 * j] = 0.f;
+      if (lane == 0) a.lse[row] = -INFINITY;
+      continue;
+    }
+    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < S; s0 += kU) {                      // splits in order
+      if (s0 % 32 == 0 && s0 > 0) {                          // next 32 splits' m and l
+        mv = s0 + lane < S ? __ldcg(pm + s0 + lane) : -INFINITY;
+        lv = s0 + lane < S ? __ldcg(pl + s0 + lane) : 0.f;
+      }
+      const float fv = (mv == -INFINITY) ? 0.f : expf(mv - M);
+      float y[kU][4];
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[u][j] = x[u][j];
+      if (s0 + kU < S) load_o(s0 + kU);                       // the next group, in flight
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (s0 + u < S) {
+          const int src = (s0 + u) & 31;
+          const float f = __shfl_sync(0xffffffffu, fv, src);
+          L = fmaf(__shfl_sync(0xffffffffu, lv, src), f, L);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[j] = fmaf(y[u][j], f, acc[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) orow[32 * j] = acc[j] / L;
+    if (lane == 0) a.lse[row] = M + logf(L);
+  }
+  if (threadIdx.x == 0) atomicExch(ctr, 0);
+}
 
 // Launchers (defined next to their kernels).  Return cudaSuccess or the launch error.
 cudaError_t launch_qtable(const cvq_shape& s, const void* q, int q_dtype, const float* key_cb,

@@ -128,6 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
       a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
       a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
     }
+    if (a.counters != nullptr) merge_tail(a, b, h, hq0, kHeads, 2 * a.n_splits);
     return;
   }
 
@@ -394,6 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     }
   }
   cluster.sync();   // no CTA leaves while its peer may still address its shared memory
+  if (a.counters != nullptr) merge_tail(a, b, h, hq0, kHeads, 2 * a.n_splits);
 }
 
 template <int R>

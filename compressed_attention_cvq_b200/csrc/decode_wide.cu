@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
       a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
       a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
     }
+    if (a.counters != nullptr) merge_tail(a, b, h, hq0, kWHeads, C * a.n_splits);
     return;
   }
 
@@ -335,6 +336,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = l_s[tid];
   }
   cluster_sync_all();          // keep oslice alive until the peer has read it
+  if (a.counters != nullptr) merge_tail(a, b, h, hq0, kWHeads, C * a.n_splits);
 }
 
 }  // namespace

@@ -175,6 +175,31 @@ CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, in
                                float* part_m, float* part_l, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * cvq_attend -- one decode step in one launch: cvq_decode_attn_gqa with the merge of
+ * cvq_combine fused into its end.  Each CTA of a work unit (sequence, KV head) counts
+ * itself in after writing its partial states; the CTA that arrives last merges the
+ * unit's query heads into out and lse (the arithmetic of cvq_combine, in the same order,
+ * so the results equal decode + combine bit for bit) and resets the unit's counter.  No
+ * CTA waits for another.
+ *
+ *   Inputs as in cvq_decode_attn_gqa (both group sizes); out [B, Hq, 128] and lse
+ *   [B, Hq] as in cvq_combine.
+ *   workspace  cvq_attend_workspace_bytes(shape, n_splits) bytes of device memory,
+ *              16-byte aligned, owned by the caller: the split partial states followed
+ *              by one int32 arrival counter per (sequence, head).  The counters must be
+ *              zero before the first call (clear the workspace once after allocating
+ *              it); every call leaves them zero.  Calls that share a workspace must be
+ *              ordered on one stream.
+ * ------------------------------------------------------------------------------- */
+CVQ_API size_t cvq_attend_workspace_bytes(const cvq_shape* shape, int n_splits);
+CVQ_API cvq_status cvq_attend(const cvq_shape* shape, const void* q, int q_dtype,
+                              const float* key_cb, int64_t key_cb_head_stride,
+                              const uint8_t* key_codes, const uint8_t* val_codes,
+                              const int32_t* seq_lens, const float* val_cb,
+                              int64_t val_cb_head_stride, int n_splits, void* workspace,
+                              float* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * cvq_combine -- merge split partial states (log-sum-exp):
  *   M = max_s m_s;  L = sum_s l_s e^{m_s - M};
  *   out[b, hq, :] = sum_s o_s e^{m_s - M} / L;   lse[b, hq] = M + ln L.

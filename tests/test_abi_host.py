@@ -205,3 +205,23 @@ def test_wide_layout_validation():
     assert b.lib.cvq_partials_bytes(ctypes.byref(_shape(**w)), 3) == 32 * 3 * 130 * 4
     assert b.lib.cvq_suggest_splits(ctypes.byref(_shape(**dict(w, t_cap=131072))), 148) == 9
     assert b.lib.cvq_suggest_splits(ctypes.byref(_shape(**dict(w, t_cap=32768, R=21))), 148) == 9
+
+
+def test_attend_workspace_and_errors():
+    s = _shape()
+    n = b.lib.cvq_attend_workspace_bytes(ctypes.byref(s), 4)
+    assert n == 32 * 4 * 130 * 4 + 32 * 4                          # partials, then counters
+    assert b.lib.cvq_attend_workspace_bytes(ctypes.byref(_shape(batch=0)), 4) == 0
+
+    def call(shape, **kw):
+        a = dict(q=FAKE, kcb=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, vcb=FAKE, ws=FAKE, out=FAKE,
+                 lse=FAKE)
+        a.update(kw)
+        return b.lib.cvq_attend(ctypes.byref(shape), a["q"], 0, a["kcb"], 0, a["kc"], a["vc"],
+                                a["lens"], a["vcb"], 0, 4, a["ws"], a["out"], a["lse"], None)
+    assert call(s, ws=None) == 1
+    assert call(s, ws=MISALIGNED) == 3
+    assert call(s, out=MISALIGNED) == 3
+    assert call(s, lse=None) == 1
+    assert call(s, kcb=None) == 1
+    assert call(_shape(R=3)) == 4
