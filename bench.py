@@ -87,20 +87,26 @@ def append_summary(w: workloads.Workload, enc_ms):
 
 def recorded_traffic(workload: str, form: str):
     """DRAM bytes per launch of the decode kernel from the committed ncu record, if it was
-    taken on this workload and the kernel source has not changed since (else None)."""
+    taken on this workload and form and none of the kernel's sources has changed since
+    (else None)."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if form not in ("gqa", "gqa_split") or not os.path.exists(path):
+    if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, rec["source"])
-    if rec.get("workload") != workload or not os.path.exists(src):
+    if rec.get("workload") != workload or rec.get("form", "gqa") != form:
         return None
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        p = os.path.join(ROOT, src)
+        if not os.path.exists(p):
             return None
+        with open(p, "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
     return float(rec["dram_bytes_per_launch"])
 
 
