@@ -34,6 +34,8 @@ CASES = [
     (8, 1, 8, 512, [512, 500, 0], 2),
     (4, 11, 64, 1024, [1024, 300, 0], 4),
     (4, 21, 64, 768, [768, 129, 5], 3),
+    (4, 1, 8, 4480, [4480, 2100, 64], 70),   # more than 32 splits: the merge reloads m, l
+    (1, 2, 8, 2112, [2112, 2049, 0], 33),
 ]
 
 
