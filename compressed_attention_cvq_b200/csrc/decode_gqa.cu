@@ -246,8 +246,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
           kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
           kw[2] = make_float2(hi.x, hi.y); kw[3] = make_float2(hi.z, hi.w);
         } else {
-          kw[0].x += lo.x; kw[0].y += lo.y; kw[1].x += lo.z; kw[1].y += lo.w;
-          kw[2].x += hi.x; kw[2].y += hi.y; kw[3].x += hi.z; kw[3].y += hi.w;
+          kw[0] = __fadd2_rn(kw[0], make_float2(lo.x, lo.y));
+          kw[1] = __fadd2_rn(kw[1], make_float2(lo.z, lo.w));
+          kw[2] = __fadd2_rn(kw[2], make_float2(hi.x, hi.y));
+          kw[3] = __fadd2_rn(kw[3], make_float2(hi.z, hi.w));
         }
       }
       float2 part2[kHeads];

@@ -203,9 +203,9 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 #pragma unroll 1
     for (int step = 0; step < kWSteps; ++step) {
       const int tt = step * kWSlots + tt0;
-      float acc[8];
+      float2 acc[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
       if (t_tile + tt < t_end) {
 #pragma unroll
         for (int r = 0; r < kRC; ++r) {
@@ -213,15 +213,17 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
             const int c = kcode[r * kWTile + tt] & (kWideCodes - 1);
             const float4* cwp = cw_s + (r * kWideCodes + c) * kWChunks;
             const float4 x = cwp[k], y = cwp[8 + k];
-            acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
-            acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+            acc[0] = __fadd2_rn(acc[0], make_float2(x.x, x.y));
+            acc[1] = __fadd2_rn(acc[1], make_float2(x.z, x.w));
+            acc[2] = __fadd2_rn(acc[2], make_float2(y.x, y.y));
+            acc[3] = __fadd2_rn(acc[3], make_float2(y.z, y.w));
           }
         }
       }
       float P[kWHeads] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        const float xr = acc[2 * p], xi = acc[2 * p + 1];
+        const float xr = acc[p].x, xi = acc[p].y;
         const float zr = fmaf(ph[p].x, xr, -ph[p].y * xi);
         const float zi = fmaf(ph[p].x, xi, ph[p].y * xr);
 #pragma unroll
