@@ -50,7 +50,9 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
       a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
       a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
     }
-    if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+    if constexpr (!TABLE) {   // the fused merge serves cvq_attend (GQA form) only
+      if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+    }
     return;
   }
 
@@ -194,7 +196,9 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
     }
     a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + dim] = acc;
   }
-  if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+  if constexpr (!TABLE) {
+    if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+  }
 }
 
 template <int NG, int R, bool TABLE>
