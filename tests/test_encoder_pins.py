@@ -78,3 +78,55 @@ def test_planted_argmax_is_caught(monkeypatch):
     monkeypatch.setattr(E, "_dist32", lambda x, c: -orig(x, c))
     with pytest.raises(AssertionError):
         test_exact_recovery_of_codeword_sums(1)
+
+
+# ---------------------------------------------------------------------------
+# the paper's layout: 2 groups of 64 scalars, 64 codewords per (group, round)
+# ---------------------------------------------------------------------------
+def _wide_cb(rng, R, scales, key=True):
+    shape = (2, 2, R, 64, 32, 2) if key else (2, 2, R, 64, 64)
+    cb = rng.standard_normal(shape).astype(np.float32)
+    for r in range(R):
+        cb[:, :, r] *= np.float32(scales[r])
+    return cb
+
+
+def test_wide_exact_recovery_of_codeword_sums():
+    """Codeword sums with rounds of decreasing scale (1, 1e-3, 1e-6) encode back to their
+    codes: each round's nearest codeword is the one that was added."""
+    rng = np.random.default_rng(11)
+    R = 3
+    kcb, vcb = _wide_cb(rng, R, (1.0, 1e-3, 1e-6)), _wide_cb(rng, R, (1.0, 1e-3, 1e-6), key=False)
+    codes = rng.integers(0, 64, size=(R, 2)).astype(np.uint8)
+    k = O.decode_keys(kcb[0], codes[None])[0].astype(np.float32)
+    v = O.decode_values(vcb[1], codes[None])[0].astype(np.float32)
+    assert np.array_equal(E.encode_vector(k, kcb[0]), codes)
+    assert np.array_equal(E.encode_vector(v, vcb[1]), codes)
+
+
+def test_wide_each_round_picks_the_nearest_codeword():
+    rng = np.random.default_rng(12)
+    cb = rng.standard_normal((11, 64, 64)).astype(np.float32) * np.float32(0.3)
+    for _ in range(20):
+        x = rng.standard_normal(64).astype(np.float32)
+        codes, _ = E.encode_group(x, cb)
+        res = x.astype(np.float64)
+        for r, c in enumerate(codes):
+            d = ((res[None, :] - cb[r].astype(np.float64)) ** 2).sum(axis=1)
+            assert d[c] <= d.min() + 1e-5 * (1 + d.min())
+            res = res - cb[r, c]
+
+
+def test_wide_append_planar_positions():
+    rng = np.random.default_rng(13)
+    kcb, vcb = _wide_cb(rng, 2, (1.0, 0.3)), _wide_cb(rng, 2, (1.0, 0.3), key=False)
+    keys = rng.standard_normal((2, 2, 128)).astype(np.float32)
+    vals = rng.standard_normal((2, 2, 128)).astype(np.float32)
+    kc = np.full((2, 2, 2, 2, 16), 99, np.uint8)        # [B, Hkv, NG, R, T_cap]
+    vc = np.full((2, 2, 2, 2, 16), 99, np.uint8)
+    E.encode_append(keys, vals, kcb, vcb, np.array([5, 16]), kc, vc, codes_layout="planar")
+    assert np.array_equal(kc[0, 1, :, :, 5], E.encode_vector(keys[0, 1], kcb[1]).T)
+    assert np.array_equal(vc[0, 0, :, :, 5], E.encode_vector(vals[0, 0], vcb[0]).T)
+    assert np.all(kc[1] == 99) and np.all(vc[1] == 99)   # position 16 >= T_cap: skipped
+    assert np.all(kc[0, :, :, :, :5] == 99) and np.all(kc[0, :, :, :, 6:] == 99)
+    assert int(kc[0, :, :, :, 5].max()) < 64
