@@ -358,7 +358,6 @@ cvq_status cvq_encode_append(const cvq_shape* s, const float* keys, const float*
                              int64_t val_cb_head_stride, const int32_t* positions,
                              uint8_t* key_codes, uint8_t* val_codes, void* stream) {
   CVQ_TRY(check_shape(s));
-  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(keys));
   CVQ_TRY(check_ptr(values));
   CVQ_TRY(check_ptr(key_cb));

@@ -1,5 +1,6 @@
 // cvq_encode_append: write the codes of one new key and value per (sequence, KV head) at
-// position positions[b] of the code cache -- the write side of a decode step.
+// position positions[b] of the code cache -- the write side of a decode step, for both
+// cache layouts (16 groups of 8 scalars; 2 groups of 64 scalars).
 //
 // The pages encode with a learned encoder (CommVQ abstract; summary page "Approach"),
 // which needs trained weights; this is greedy additive quantization instead: for each
@@ -94,12 +95,87 @@ __global__ void __launch_bounds__(32 * kEncWarps) encode_kernel(
   }
 }
 
+// The paper's layout: 2 groups of 64 scalars, 64 codewords per (group, round), planar codes
+// [B, Hkv, 2, R, t_cap].  One warp per (sequence x KV head, key | value, group); lane l scores
+// codewords l and l + 32.  The residual (64 floats) sits in shared memory and every lane
+// reads it in dim order 0..63, so each distance is summed in one fixed order.
+constexpr int kWideEncWarps = 8;
+
+__global__ void __launch_bounds__(32 * kWideEncWarps) encode_wide_kernel(
+    const float* __restrict__ keys, const float* __restrict__ values,
+    const float* __restrict__ key_cb, long long key_stride, const float* __restrict__ val_cb,
+    long long val_stride, const int32_t* __restrict__ positions, uint8_t* __restrict__ key_codes,
+    uint8_t* __restrict__ val_codes, int R, int n_kv_heads, int t_cap, int n_units) {
+  __shared__ __align__(16) float res_s[kWideEncWarps][kWideVDims];
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int unit = blockIdx.x * kWideEncWarps + wl;             // (bh, is_val, G)
+  if (unit >= n_units) return;                                   // uniform for the warp
+  const int G = unit & 1, is_val = (unit >> 1) & 1, bh = unit >> 2;
+  const int b = bh / n_kv_heads, h = bh % n_kv_heads;
+  const int p = positions[b];
+  if (p < 0 || p >= t_cap) return;                               // uniform for the warp
+  const float* src = (is_val ? values : keys) + static_cast<size_t>(bh) * kHeadDim + kWideVDims * G;
+  const float* cb = (is_val ? val_cb + h * val_stride : key_cb + h * key_stride) +
+                    static_cast<size_t>(G) * R * kWideCodes * kWideVDims;
+  uint8_t* out = (is_val ? val_codes : key_codes) +
+                 ((static_cast<size_t>(bh) * kWideGroups + G) * R) * t_cap + p;
+  float* res = res_s[wl];
+  res[lane] = src[lane];
+  res[lane + 32] = src[lane + 32];
+  __syncwarp();
+  for (int r = 0; r < R; ++r) {
+    const float4* c0 = reinterpret_cast<const float4*>(cb + (static_cast<size_t>(r) * kWideCodes + lane) * kWideVDims);
+    const float4* c1 = c0 + 32 * kWideVDims / 4;                 // codeword lane + 32
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < kWideVDims / 4; ++q) {
+      const float4 x0 = __ldg(c0 + q), x1 = __ldg(c1 + q);
+      const float4 rv = *reinterpret_cast<const float4*>(res + 4 * q);
+      float d;
+      d = __fsub_rn(rv.x, x0.x); a0 = __fadd_rn(a0, __fmul_rn(d, d));
+      d = __fsub_rn(rv.y, x0.y); a0 = __fadd_rn(a0, __fmul_rn(d, d));
+      d = __fsub_rn(rv.z, x0.z); a0 = __fadd_rn(a0, __fmul_rn(d, d));
+      d = __fsub_rn(rv.w, x0.w); a0 = __fadd_rn(a0, __fmul_rn(d, d));
+      d = __fsub_rn(rv.x, x1.x); a1 = __fadd_rn(a1, __fmul_rn(d, d));
+      d = __fsub_rn(rv.y, x1.y); a1 = __fadd_rn(a1, __fmul_rn(d, d));
+      d = __fsub_rn(rv.z, x1.z); a1 = __fadd_rn(a1, __fmul_rn(d, d));
+      d = __fsub_rn(rv.w, x1.w); a1 = __fadd_rn(a1, __fmul_rn(d, d));
+    }
+    // arg-min over (distance, code): this lane's two, then the warp
+    float bd = a0;
+    int bc = lane;
+    if (a1 < bd) { bd = a1; bc = lane + 32; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+      const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+      if (od < bd || (od == bd && oc < bc)) { bd = od; bc = oc; }
+    }
+    if (lane == 0) out[static_cast<size_t>(r) * t_cap] = static_cast<uint8_t>(bc);
+    const float* chosen = cb + (static_cast<size_t>(r) * kWideCodes + bc) * kWideVDims;
+    const float n0 = __fsub_rn(res[lane], __ldg(chosen + lane));
+    const float n1 = __fsub_rn(res[lane + 32], __ldg(chosen + lane + 32));
+    __syncwarp();                                                // every lane read res
+    res[lane] = n0;
+    res[lane + 32] = n1;
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const float* values,
                                  const float* key_cb, long long key_stride, const float* val_cb,
                                  long long val_stride, const int32_t* positions,
                                  uint8_t* key_codes, uint8_t* val_codes, cudaStream_t stream) {
+  if (s.group_dim == kWideGroupDim) {
+    const int n_units = s.batch * s.n_kv_heads * 2 * kWideGroups;
+    const unsigned blocks = static_cast<unsigned>((n_units + kWideEncWarps - 1) / kWideEncWarps);
+    encode_wide_kernel<<<blocks, 32 * kWideEncWarps, 0, stream>>>(
+        keys, values, key_cb, key_stride, val_cb, val_stride, positions, key_codes, val_codes,
+        s.R, s.n_kv_heads, s.t_cap, n_units);
+    return cudaGetLastError();
+  }
   // units = B * Hkv * 2 * 16, a multiple of kEncWarps
   const unsigned blocks = static_cast<unsigned>(s.batch) * s.n_kv_heads * 32 / kEncWarps;
   encode_kernel<<<blocks, 32 * kEncWarps, 0, stream>>>(keys, values, key_cb, key_stride, val_cb,

@@ -248,12 +248,15 @@ CVQ_API cvq_status cvq_naive_decode(const cvq_shape* shape, const void* q, int q
  *
  *   keys, values  [B, Hkv, 128] fp32 (16-byte aligned); a key group G is its pairs
  *                 4G..4G+3 as dims 8G..8G+7 (re, im interleaved), a value group G is
- *                 dims 8G..8G+7
+ *                 dims 8G..8G+7 (with group_dim = 64: pairs 32G..32G+31 and dims
+ *                 64G..64G+63, 64 codewords per (group, round), distances summed over
+ *                 the 64 dims in order)
  *   key_cb, val_cb and their head strides as in cvq_decode_attn_gqa
  *   positions     [B] int32 (device): the token index t each sequence writes; an index
  *                 outside [0, t_cap) writes nothing for that sequence
  *   key_codes, val_codes  [B, Hkv, t_cap, R, 16] uint8, written at [b, h, positions[b]]
- *                 and nowhere else (the caller owns them; seq_lens is the caller's to
+ *                 (group_dim = 64: planar [B, Hkv, 2, R, t_cap], written at
+ *                 [b, h, :, :, positions[b]]) and nowhere else (the caller owns them; seq_lens is the caller's to
  *                 advance)
  *   Errors: CVQ_ERR_NULL / CVQ_ERR_ALIGN / CVQ_ERR_SHAPE / CVQ_ERR_UNSUPPORTED before any
  *   launch; CVQ_ERR_CUDA if the launch fails.  Asynchronous on `stream`.

@@ -200,7 +200,8 @@ def test_wide_layout_validation():
     assert _gqa(_shape(group_dim=32)) == 4
     assert _qtable(_shape(**w)) == 4
     assert _decode(_shape(**w)) == 4
-    assert _encode(_shape(**w)) == 4
+    assert _encode(_shape(**w), kc=None) == 1                        # the encoder takes it
+    assert _encode(_shape(**w), vstride=8192 * 11 + 2) == 3
     assert b.lib.cvq_ptable_bytes(ctypes.byref(_shape(**w))) == 0
     assert b.lib.cvq_partials_bytes(ctypes.byref(_shape(**w)), 3) == 32 * 3 * 130 * 4
     assert b.lib.cvq_suggest_splits(ctypes.byref(_shape(**dict(w, t_cap=131072))), 148) == 9

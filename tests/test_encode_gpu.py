@@ -141,3 +141,55 @@ def test_full_size_batch16():
     keys, vals = _new_vectors(rng, d, True)
     gk, gv, ok, ov = _run(d, keys, vals, d["seq_lens"])
     assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+
+
+# ---------------------------------------------------------------------------
+# the paper's layout: 2 groups of 64 scalars, 64 codewords, planar codes [B, Hkv, 2, R, T]
+# ---------------------------------------------------------------------------
+def _wide_case(R, T, lens, seed):
+    return workloads.small(batch=len(lens), n_q_heads=8, n_kv_heads=2, t_cap=T, R=R,
+                           seq_lens=np.asarray(lens, np.int32), seed=seed,
+                           cb_std=math.sqrt(1.0 / R), group_dim=64)
+
+
+@pytest.mark.parametrize("R", [1, 11, 21])
+def test_wide_codes_bit_exact(R):
+    d = _wide_case(R, 48, [48, 48, 48], seed=80 + R)
+    rng = np.random.default_rng(800 + R)
+    keys = rng.standard_normal((3, 2, 128), dtype=np.float32)
+    vals = rng.standard_normal((3, 2, 128), dtype=np.float32)
+    positions = np.array([0, 47, -3], np.int32)
+    kc = np.full(d["key_codes"].shape, FILL, np.uint8)
+    vc = np.full(d["val_codes"].shape, FILL, np.uint8)
+    dk, dv = torch.from_numpy(kc.copy()).cuda(), torch.from_numpy(vc.copy()).cuda()
+    shape = cvq.make_shape(3, 8, 2, R, 48, d["rope_base"], 128, 64)
+    cvq.encode_append(shape, torch.from_numpy(keys).cuda(), torch.from_numpy(vals).cuda(),
+                      torch.from_numpy(d["key_cb"]).cuda(), torch.from_numpy(d["val_cb"]).cuda(),
+                      torch.from_numpy(positions).cuda(), dk, dv)
+    torch.cuda.synchronize()
+    E.encode_append(keys, vals, d["key_cb"], d["val_cb"], positions, kc, vc, codes_layout="planar")
+    gk, gv = dk.cpu().numpy(), dv.cpu().numpy()
+    assert np.array_equal(gk, kc) and np.array_equal(gv, vc)
+    assert np.all(gk[2] == FILL) and int(gk[0, :, :, :, 0].max()) < 64
+
+
+def test_wide_append_then_attend_matches_oracle():
+    d = _wide_case(11, 512, [300, 511], seed=85)
+    rng = np.random.default_rng(85)
+    keys = rng.standard_normal((2, 2, 128), dtype=np.float32)
+    vals = rng.standard_normal((2, 2, 128), dtype=np.float32)
+    dd = to_device(d)
+    shape = cvq.shape_of(dd["q"], dd["key_codes"], d["rope_base"], 64)
+    cvq.encode_append(shape, torch.from_numpy(keys).cuda(), torch.from_numpy(vals).cuda(),
+                      dd["key_cb"], dd["val_cb"], dd["seq_lens"].clone(), dd["key_codes"],
+                      dd["val_codes"])
+    dd["seq_lens"] += 1
+    kc, vc = d["key_codes"].copy(), d["val_codes"].copy()
+    E.encode_append(keys, vals, d["key_cb"], d["val_cb"], d["seq_lens"], kc, vc,
+                    codes_layout="planar")
+    d2 = dict(d, key_codes=kc, val_codes=vc, seq_lens=d["seq_lens"] + 1)
+    assert np.array_equal(dd["key_codes"].cpu().numpy(), kc)
+    assert np.array_equal(dd["val_codes"].cpu().numpy(), vc)
+    out, lse = run_gpu(d2, dd=dd)
+    ref_out, ref_lse = run_oracle(d2)
+    assert_close(out, lse, ref_out, ref_lse)
