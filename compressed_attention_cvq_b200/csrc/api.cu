@@ -198,26 +198,30 @@ int32_t cvq_split_tokens(const cvq_shape* s, int n_splits) {
 int cvq_suggest_splits(const cvq_shape* s, int sm_count) {
   if (check_shape(s) != CVQ_OK || sm_count < 1) return 1;
   // CTAs per split index and CTA slots on the GPU: the 4-head kernel runs a cluster of 2
-  // CTAs per (sequence, KV head, split), 2 per SM at R = 1 and 1 per SM at R = 2; the
-  // plain kernel runs one CTA per (sequence, KV head, split).  Take the fewest splits
-  // (longest, so the per-CTA codebook load and epilogue are amortized) whose CTAs fill
-  // at least 90% of their last wave.
-  // With 64-scalar groups the kernel runs a cluster of 2 * ceil(R / 11) CTAs, one per SM.
+  // CTAs per (sequence, KV head, split), 2 per SM at R = 1 and 1 per SM at R = 2; with
+  // 64-scalar groups a cluster of 2 * ceil(R / 11) CTAs, one per SM; the plain kernel runs
+  // one CTA per (sequence, KV head, split).  Every split of a launch is equally long, so a
+  // launch takes about waves x (split length + a fixed cost per CTA for loading the
+  // codebooks and the epilogue, ~min_len tokens' worth); take the split count that
+  // minimizes that, the fewest splits on a tie.
   const bool clustered = (s->n_q_heads / s->n_kv_heads) == 4;
   const long long per_split = is_wide(s) ? wide_cluster_size(s->R) : (clustered ? 2 : 1);
   const long long units = static_cast<long long>(s->batch) * s->n_kv_heads * per_split;
   const long long slots =
       static_cast<long long>(sm_count) * (clustered && !is_wide(s) && s->R == 1 ? 2 : 1);
-  // the clustered kernel amortizes a 64R KiB codebook load per CTA, so its splits stay
-  // >= 256 tokens; the plain kernel's splits may be as short as one 64-token block
   const long long min_len = clustered ? 256LL : 64LL;
   const long long max_splits = std::max(1LL, std::min(4096LL, (s->t_cap + min_len - 1) / min_len));
+  long long best_n = 1, best_cost = -1;
   for (long long n = 1; n <= max_splits; ++n) {
-    const long long ctas = units * n;
-    const long long waves = (ctas + slots - 1) / slots;
-    if (ctas * 10 >= waves * slots * 9) return static_cast<int>(n);
+    const long long waves = (units * n + slots - 1) / slots;
+    const long long len = split_tokens_host(s->t_cap, static_cast<int>(n));
+    const long long cost = waves * (len + min_len);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_n = n;
+    }
   }
-  return static_cast<int>(max_splits);
+  return static_cast<int>(best_n);
 }
 
 cvq_status cvq_qtable(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
