@@ -125,7 +125,8 @@ CVQ_API cvq_status cvq_qtable(const cvq_shape* shape, const void* q, int q_dtype
  * ------------------------------------------------------------------------------- */
 CVQ_API size_t cvq_partials_bytes(const cvq_shape* shape, int n_splits);
 CVQ_API int32_t cvq_split_tokens(const cvq_shape* shape, int n_splits);
-/* A split count that fills `sm_count` SMs for this shape (a suggestion). */
+/* A split count for this shape on `sm_count` SMs (a suggestion): the count that minimizes
+   waves x (split length + a fixed per-CTA cost), the fewest on a tie. */
 CVQ_API int cvq_suggest_splits(const cvq_shape* shape, int sm_count);
 
 /* ---------------------------------------------------------------------------------
