@@ -318,7 +318,6 @@ cvq_status cvq_naive_dequant(const cvq_shape* s, const float* key_cb, int64_t ke
                              const int32_t* seq_lens, const float* val_cb,
                              int64_t val_cb_head_stride, void* k_out, void* v_out, void* stream) {
   CVQ_TRY(check_shape(s));
-  if (is_wide(s)) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(key_cb));
   CVQ_TRY(check_ptr(val_cb));
   CVQ_TRY(check_ptr(key_codes));

@@ -7,7 +7,8 @@
 // naive_dequant_kernel: one thread per (token, group); the thread sums the R key codewords
 // of its 4 pairs, rotates them by the exact phase of position t and stores 8 fp16 key dims,
 // then sums the R value codewords and stores 8 fp16 value dims.
-// The attention half is naive_decode.cu.
+// The attention half is naive_decode.cu; naive_dequant_wide_kernel below does the paper's
+// layout.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -60,6 +61,54 @@ __global__ void __launch_bounds__(kDqThreads) naive_dequant_kernel(
   *reinterpret_cast<uint4*>(v_out + row * kHeadDim + 8 * G) = *reinterpret_cast<uint4*>(vo);
 }
 
+// The same for the paper's layout (2 groups of 64 scalars, 64 codewords, planar codes
+// [B, Hkv, 2, R, t_cap]): block (32 tokens, 8 chunks) per (token block, KV head x group,
+// sequence); thread (token, chunk) sums the R codewords' 8-float chunk of its group for
+// the key (pairs 32 G + 4 chunk .. + 3, rotated) and the value (dims 64 G + 8 chunk ..).
+__global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
+    const float* __restrict__ key_cb, long long key_stride, const float* __restrict__ val_cb,
+    long long val_stride, const uint8_t* __restrict__ key_codes,
+    const uint8_t* __restrict__ val_codes, const int32_t* __restrict__ seq_lens, int R,
+    int n_kv_heads, int t_cap, PhaseTurns phase, __half* __restrict__ k_out,
+    __half* __restrict__ v_out) {
+  const int t = blockIdx.x * 32 + threadIdx.x;
+  const int chunk = threadIdx.y;
+  const int G = blockIdx.y & 1, h = blockIdx.y >> 1, b = blockIdx.z;
+  int L = seq_lens[b];
+  L = L < 0 ? 0 : (L > t_cap ? t_cap : L);
+  if (t >= L) return;
+  const size_t bh = static_cast<size_t>(b) * n_kv_heads + h;
+  const uint8_t* kc = key_codes + (bh * kWideGroups + G) * R * static_cast<size_t>(t_cap) + t;
+  const uint8_t* vc = val_codes + (bh * kWideGroups + G) * R * static_cast<size_t>(t_cap) + t;
+  const float* kcb = key_cb + h * key_stride + static_cast<size_t>(G) * R * kWideCodes * kWideVDims + 8 * chunk;
+  const float* vcb = val_cb + h * val_stride + static_cast<size_t>(G) * R * kWideCodes * kWideVDims + 8 * chunk;
+  float k[8], v[8];
+#pragma unroll
+  for (int d = 0; d < 8; ++d) k[d] = v[d] = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const int ck = kc[static_cast<size_t>(r) * t_cap] & (kWideCodes - 1);
+    const int cv = vc[static_cast<size_t>(r) * t_cap] & (kWideCodes - 1);
+    const float4* kw = reinterpret_cast<const float4*>(kcb + (static_cast<size_t>(r) * kWideCodes + ck) * kWideVDims);
+    const float4* vw = reinterpret_cast<const float4*>(vcb + (static_cast<size_t>(r) * kWideCodes + cv) * kWideVDims);
+    const float4 a0 = __ldg(kw), a1 = __ldg(kw + 1), b0 = __ldg(vw), b1 = __ldg(vw + 1);
+    k[0] += a0.x; k[1] += a0.y; k[2] += a0.z; k[3] += a0.w;
+    k[4] += a1.x; k[5] += a1.y; k[6] += a1.z; k[7] += a1.w;
+    v[0] += b0.x; v[1] += b0.y; v[2] += b0.z; v[3] += b0.w;
+    v[4] += b1.x; v[5] += b1.y; v[6] += b1.z; v[7] += b1.w;
+  }
+  __half2 ko[4], vo[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float2 ph = phase_at(phase.F[kWidePairs * G + 4 * chunk + p], t);
+    ko[p] = __floats2half2_rn(ph.x * k[2 * p] - ph.y * k[2 * p + 1],
+                              ph.y * k[2 * p] + ph.x * k[2 * p + 1]);
+    vo[p] = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
+  }
+  const size_t o = (bh * t_cap + t) * kHeadDim + kWideVDims * G + 8 * chunk;
+  *reinterpret_cast<uint4*>(k_out + o) = *reinterpret_cast<uint4*>(ko);
+  *reinterpret_cast<uint4*>(v_out + o) = *reinterpret_cast<uint4*>(vo);
+}
+
 }  // namespace
 
 cudaError_t launch_naive_dequant(const cvq_shape& s, const float* key_cb, long long key_stride,
@@ -68,6 +117,13 @@ cudaError_t launch_naive_dequant(const cvq_shape& s, const float* key_cb, long l
                                  const int32_t* seq_lens, const PhaseTurns& phase, void* k_out,
                                  void* v_out, cudaStream_t stream) {
   if (s.t_cap == 0) return cudaSuccess;
+  if (s.group_dim == kWideGroupDim) {
+    dim3 grid((s.t_cap + 31) / 32, s.n_kv_heads * kWideGroups, s.batch);
+    naive_dequant_wide_kernel<<<grid, dim3(32, 8), 0, stream>>>(
+        key_cb, key_stride, val_cb, val_stride, key_codes, val_codes, seq_lens, s.R,
+        s.n_kv_heads, s.t_cap, phase, static_cast<__half*>(k_out), static_cast<__half*>(v_out));
+    return cudaGetLastError();
+  }
   dim3 grid((s.t_cap + kDqThreads / 16 - 1) / (kDqThreads / 16), s.n_kv_heads, s.batch);
   naive_dequant_kernel<<<grid, kDqThreads, 0, stream>>>(
       key_cb, key_stride, val_cb, val_stride, key_codes, val_codes, seq_lens, s.R, s.n_kv_heads,

@@ -25,8 +25,8 @@
  *   score_t = sum_j Re(e^{i theta_j t} conj(q_j) sum_r c_{t,r,j}) / sqrt(128), t = 0..L-1
  *   out = sum_t softmax(score)_t v_t,   lse = ln sum_t exp(score_t).
  * Query head hq reads KV head hq / (n_q_heads / n_kv_heads).
- * Every entry point takes g = 8; cvq_decode_attn_gqa (4 query heads per KV head),
- * cvq_attend_static, cvq_combine and the size helpers also take g = 64; the others
+ * Every entry point takes g = 8; all but cvq_qtable and cvq_decode_attn (the table
+ * form) also take g = 64 (the GQA decode with 4 query heads per KV head), and those two
  * return CVQ_ERR_UNSUPPORTED for it.
  *
  * Conventions for every call:

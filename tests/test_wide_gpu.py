@@ -136,13 +136,43 @@ def test_wide_static_entry():
                  ref_out, ref_lse)
 
 
-def test_wide_unsupported_forms_fail_loudly():
+def test_wide_table_form_fails_loudly():
     d = _wide(256, 11, [256, 256], seed=75)
     dd = to_device(d)
     with pytest.raises(cvq.CvqError):
         run_gpu(d, form="table", dd=dd)
-    with pytest.raises(cvq.CvqError):
-        run_gpu(d, form="naive", dd=dd)
+
+
+@pytest.mark.parametrize("R", [3, 11, 21])
+def test_wide_naive_dequant_matches_oracle(R):
+    """The naive comparison path in the paper's layout: every cached key (rotated by RoPE)
+    and value decoded into fp16 equals the oracle's reconstruction to fp16 rounding."""
+    lens = np.array([200, 77], np.int32)
+    d = _wide(208, R, lens, seed=76 + R)
+    dd = to_device(d)
+    shape = cvq.shape_of(dd["q"], dd["key_codes"], d["rope_base"], 64)
+    k, v = cvq.naive_dequant(shape, dd["key_cb"], dd["val_cb"], dd["key_codes"], dd["val_codes"],
+                             dd["seq_lens"])
+    torch.cuda.synchronize()
+    k, v = k.float().cpu().numpy(), v.float().cpu().numpy()
+    theta = O.rope_theta(d["rope_base"])
+    kt, vt = O.token_major(d["key_codes"]), O.token_major(d["val_codes"])
+    for b in range(2):
+        for h in range(2):
+            L = int(lens[b])
+            rk = O.apply_rope(O.decode_keys(d["key_cb"][h], kt[b, h, :L]), np.arange(L), theta)
+            vv = O.decode_values(d["val_cb"][h], vt[b, h, :L])
+            np.testing.assert_allclose(k[b, h, :L], rk, rtol=2 ** -10, atol=1e-5)
+            np.testing.assert_allclose(v[b, h, :L], vv, rtol=2 ** -10, atol=1e-6)
+            assert np.all(k[b, h, L:] == 0) and np.all(v[b, h, L:] == 0)
+
+
+@pytest.mark.parametrize("R,T", [(11, 1024), (21, 512)])
+def test_wide_naive_attention_matches_oracle(R, T):
+    d = _wide(T, R, [T, T // 3 + 5], seed=78 + R)
+    out, lse = run_gpu(d, form="naive", n_splits=3)
+    ref_out, ref_lse = run_oracle(d)
+    assert_close(out, lse, ref_out, ref_lse)
 
 
 @pytest.mark.parametrize("name,k", [("llama8b_layer_T131072_R11_g64", 3),
