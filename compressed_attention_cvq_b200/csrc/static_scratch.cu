@@ -1,5 +1,6 @@
-// cvq_attend_static: one decode step (GQA decode + combine) whose split partial states
-// live in a fixed, file-scope device array instead of caller-allocated memory.
+// cvq_attend_static: one decode step (the GQA decode with the fused split merge,
+// cvq_attend) whose workspace -- split partial states and arrival counters -- is a fixed,
+// file-scope device array instead of caller-allocated memory.
 //
 // For callers that cannot allocate device memory while decoding: a serving process whose
 // memory pool has already claimed all free HBM for the KV cache, a plugin whose host
@@ -57,20 +58,17 @@ extern "C" CVQ_API cvq_status cvq_attend_static(
   if (s == nullptr) return CVQ_ERR_NULL;
   if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
   if (s->batch < 1 || s->n_q_heads < 1) return CVQ_ERR_SHAPE;
-  const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
-  if (rows * (kHeadDim + 2) > kStaticScratchFloats) return CVQ_ERR_STATIC_LIMIT;
+  const size_t need = cvq_attend_workspace_bytes(s, n_splits);
+  if (need == 0)   // an invalid shape: cvq_attend reports which check fails, before any launch
+    return cvq_attend(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes, seq_lens,
+                      val_cb, val_cb_head_stride, n_splits, nullptr, out, lse, stream);
+  if (need > CVQ_STATIC_SCRATCH_BYTES) return CVQ_ERR_STATIC_LIMIT;
 
   float* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return CVQ_ERR_CUDA;
-  // part_o [rows, 128], then part_m [rows], then part_l [rows]; every slot the combine
-  // reads is written by the decode of the same call, so nothing needs clearing.
-  float* part_o = base;
-  float* part_m = base + rows * kHeadDim;
-  float* part_l = part_m + rows;
-  const cvq_status st =
-      cvq_decode_attn_gqa(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
-                          seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
-                          stream);
-  if (st != CVQ_OK) return st;
-  return cvq_combine(s, n_splits, part_o, part_m, part_l, out, lse, stream);
+  // The array is cvq_attend's workspace: the split partial states, then one arrival
+  // counter per (sequence, head).  Static device memory starts zeroed and every call
+  // leaves the counters zero, so nothing needs clearing.
+  return cvq_attend(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes, seq_lens,
+                    val_cb, val_cb_head_stride, n_splits, base, out, lse, stream);
 }

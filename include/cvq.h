@@ -269,16 +269,16 @@ CVQ_API cvq_status cvq_encode_append(const cvq_shape* shape, const float* keys, 
                                      uint8_t* val_codes, void* stream);
 
 /* ---------------------------------------------------------------------------------
- * cvq_attend_static -- cvq_decode_attn_gqa followed by cvq_combine, with the split
- * partial states kept in a fixed device array inside the library instead of memory
- * the caller allocates.  The paper has no counterpart: this is an interface for
+ * cvq_attend_static -- cvq_attend (decode with the fused split merge, one launch) with
+ * its workspace -- the split partial states and the arrival counters -- kept in a fixed
+ * device array inside the library instead of memory the caller allocates.  The paper has no counterpart: this is an interface for
  * callers that cannot allocate device memory while decoding -- a serving process
  * whose pool has already claimed all free HBM for the KV cache, a plugin whose host
  * gives it no allocator, or a decode loop that cannot afford cudaMalloc's implicit
  * synchronization.  The call itself allocates nothing.
  *
  *   Arguments as in cvq_decode_attn_gqa, then out [B, Hq, 128] and lse [B, Hq] as in
- *   cvq_combine.  B * Hq * n_splits * 130 * 4 bytes must fit in
+ *   cvq_combine.  cvq_attend_workspace_bytes(shape, n_splits) must fit in
  *   CVQ_STATIC_SCRATCH_BYTES (4 MiB, held by every GPU that loads the library until
  *   the process exits); larger calls return CVQ_ERR_STATIC_LIMIT before any launch.
  *   The first call on a device looks up the array's device address with that device

@@ -226,3 +226,13 @@ def test_attend_workspace_and_errors():
     assert call(s, lse=None) == 1
     assert call(s, kcb=None) == 1
     assert call(_shape(R=3)) == 4
+
+
+def test_static_entry_reports_shape_errors():
+    fake = FAKE
+    st = b.lib.cvq_attend_static(ctypes.byref(_shape(R=3)), fake, 0, fake, 0, fake, fake, fake,
+                                 fake, 0, 4, fake, fake, None)
+    assert st == 4
+    st = b.lib.cvq_attend_static(ctypes.byref(_shape(n_q_heads=12)), fake, 0, fake, 0, fake,
+                                 fake, fake, fake, 0, 4, fake, fake, None)
+    assert st == 2
