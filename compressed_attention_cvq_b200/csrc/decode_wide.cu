@@ -27,7 +27,9 @@
 //   bins: float r * kBinRow + c * 4 + head (kBinRow = 260, so consecutive rounds start 4
 //     banks apart);
 //   codes: [buffer][key | value][rc][256 tokens] bytes, copied with cp.async from the
-//     planar global layout [B, Hkv, 2, R, t_cap] while the previous tile computes.
+//     planar global layout [B, Hkv, 2, R, t_cap] while the previous tile computes, then
+//     transposed once per tile to [key | value][256 tokens][16 bytes] so a token's rc codes
+//     come in one 16-byte load.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -53,8 +55,9 @@ constexpr size_t kCwBytes = sizeof(float4) * kRC * kWideCodes * kWChunks;   // 1
 constexpr size_t kBinBytes = sizeof(float) * kRC * kBinRow;                 //  11,440
 constexpr size_t kXchgBytes = sizeof(float) * 2 * kWTile * kWHeads;         //   8,192
 constexpr size_t kCodeBytes = 2 * 2 * kRC * kWTile;                         //  11,264
+constexpr size_t kTCodeBytes = 2 * kWTile * 16;                              //   8,192
 constexpr size_t kRedBytes = sizeof(float) * (2 * kWWarps * kWHeads + 4 * kWHeads);
-constexpr size_t kWSmem = kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kRedBytes;
+constexpr size_t kWSmem = kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kTCodeBytes + kRedBytes;
 static_assert(kWSteps * kWSlots == kWTile, "tile must be a whole number of steps");
 static_assert(kWSmem <= 227 * 1024, "shared memory per CTA");
 
@@ -86,7 +89,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   float* bins = reinterpret_cast<float*>(smem4 + kRC * kWideCodes * kWChunks);
   float* xchg = bins + kRC * kBinRow;                                         // [2][256][4]
   uint8_t* code_s = reinterpret_cast<uint8_t*>(xchg + 2 * kWTile * kWHeads);  // [2][2][rc][256]
-  float* red_m = reinterpret_cast<float*>(code_s + kCodeBytes);              // [16][4]
+  uint8_t* tcode = code_s + kCodeBytes;                                       // [2][256][16]
+  float* red_m = reinterpret_cast<float*>(tcode + kTCodeBytes);              // [16][4]
   float* red_l = red_m + kWWarps * kWHeads;                                   // [16][4]
   float* mref_s = red_l + kWWarps * kWHeads;                                  // [4]
   float* l_s = mref_s + kWHeads;                                              // [4]
@@ -192,8 +196,18 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     __syncthreads();                          // codes of this tile (and the codebook) landed
     if (it + 1 < n_tiles) stage_codes(t_tile + kWTile, buf ^ 1);
     cp_async_commit();
-    const uint8_t* kcode = code_s + (buf * 2 + 0) * kRC * kWTile;
-    const uint8_t* vcode = code_s + (buf * 2 + 1) * kRC * kWTile;
+    // token-major copy of this tile's codes: 16 bytes per (key | value, token), byte r =
+    // round r, so one 16-byte load gives a token all its codes
+    {
+      const int kind = tid >> 8, t = tid & 255;
+      const uint8_t* src = code_s + (buf * 2 + kind) * kRC * kWTile + t;
+      uint32_t wv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int r = 0; r < kRC; ++r)
+        if (r < rc) wv[r >> 2] |= static_cast<uint32_t>(src[r * kWTile]) << (8 * (r & 3));
+      *reinterpret_cast<uint4*>(tcode + (kind * kWTile + t) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+    __syncthreads();
     float* xo = xchg + buf * kWTile * kWHeads;
 
     // ---- this CTA's share of every token's 4 scores ----
@@ -207,10 +221,12 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
       if (t_tile + tt < t_end) {
+        const uint4 kc4 = *reinterpret_cast<const uint4*>(tcode + tt * 16);
+        const uint32_t kcw[4] = {kc4.x, kc4.y, kc4.z, kc4.w};
 #pragma unroll
         for (int r = 0; r < kRC; ++r) {
           if (r < rc) {
-            const int c = kcode[r * kWTile + tt] & (kWideCodes - 1);
+            const int c = (kcw[r >> 2] >> (8 * (r & 3))) & (kWideCodes - 1);
             const float4* cwp = cw_s + (r * kWideCodes + c) * kWChunks;
             const float4 x = cwp[k], y = cwp[8 + k];
             acc[0] = __fadd2_rn(acc[0], make_float2(x.x, x.y));
@@ -288,12 +304,20 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     if (lane < kWHeads) red_l[warp * kWHeads + lane] = ls;
     // value reorder: the weight goes to the bin of the token's value code, per own round
     if (wA > 0.f) {
-      for (int r = 0; r < rc; ++r)
-        atomicAdd(&bins[r * kBinRow + (vcode[r * kWTile + tA] & (kWideCodes - 1)) * kWHeads + hh], wA);
+      const uint4 v4 = *reinterpret_cast<const uint4*>(tcode + (kWTile + tA) * 16);
+      const uint32_t vcw[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+      for (int r = 0; r < kRC; ++r)
+        if (r < rc)
+          atomicAdd(&bins[r * kBinRow + ((vcw[r >> 2] >> (8 * (r & 3))) & (kWideCodes - 1)) * kWHeads + hh], wA);
     }
     if (wB > 0.f) {
-      for (int r = 0; r < rc; ++r)
-        atomicAdd(&bins[r * kBinRow + (vcode[r * kWTile + tB] & (kWideCodes - 1)) * kWHeads + hh], wB);
+      const uint4 v4 = *reinterpret_cast<const uint4*>(tcode + (kWTile + tB) * 16);
+      const uint32_t vcw[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+      for (int r = 0; r < kRC; ++r)
+        if (r < rc)
+          atomicAdd(&bins[r * kBinRow + ((vcw[r >> 2] >> (8 * (r & 3))) & (kWideCodes - 1)) * kWHeads + hh], wB);
     }
   }
   __syncthreads();
