@@ -24,8 +24,9 @@
 // Layouts in shared memory (32 banks x 4 bytes):
 //   key / value codewords: [rc][64 codes][16 chunks of 16 bytes]; lane k of a token reads
 //     chunks k and 8 + k, so the 8 lanes of a quarter-warp read 128 contiguous bytes;
-//   bins: float r * kBinRow + c * 4 + head (kBinRow = 260, so consecutive rounds start 4
-//     banks apart);
+//   bins: float c * 64 + 4 r + head; a warp's 8 tokens bin 8 different rounds at each
+//     atomic step (the token's slot in the warp rotates its round order), so the 32 lanes
+//     of an atomic hit 32 different banks whatever the codes;
 //   codes: [buffer][key | value][rc][256 tokens] bytes, copied with cp.async from the
 //     planar global layout [B, Hkv, 2, R, t_cap] while the previous tile computes, then
 //     transposed once per tile to [key | value][256 tokens][16 bytes] so a token's rc codes
@@ -47,12 +48,13 @@ constexpr int kWWarps = kWThreads / 32;
 constexpr int kWSlots = kWWarps * 4;              // tokens per step
 constexpr int kWSteps = kWTile / kWSlots;         // steps per tile
 constexpr int kWChunks = kWidePairs * 2 / 4;      // 16-byte chunks per codeword (16)
-constexpr int kBinRow = kWideCodes * kWHeads + 4; // floats per round of bins (padded)
+constexpr int kBinStride = 64;                     // floats per code: 4 r + head, r < 11
 constexpr float kWSlack = 8.0f;
 constexpr int kRC = kWideRoundsPerCta;
 
 constexpr size_t kCwBytes = sizeof(float4) * kRC * kWideCodes * kWChunks;   // 180,224
-constexpr size_t kBinBytes = sizeof(float) * kRC * kBinRow;                 //  11,440
+constexpr size_t kBinBytes = sizeof(float) * kWideCodes * kBinStride;      //  16,384
+static_assert(4 * kRC <= kBinStride, "bins of one code");
 constexpr size_t kXchgBytes = sizeof(float) * 2 * kWTile * kWHeads;         //   8,192
 constexpr size_t kCodeBytes = 2 * 2 * kRC * kWTile;                         //  11,264
 constexpr size_t kTCodeBytes = 2 * kWTile * 16;                              //   8,192
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   extern __shared__ float4 smem4[];
   float4* cw_s = smem4;                                                       // codewords
   float* bins = reinterpret_cast<float*>(smem4 + kRC * kWideCodes * kWChunks);
-  float* xchg = bins + kRC * kBinRow;                                         // [2][256][4]
+  float* xchg = bins + kWideCodes * kBinStride;                               // [2][256][4]
   uint8_t* code_s = reinterpret_cast<uint8_t*>(xchg + 2 * kWTile * kWHeads);  // [2][2][rc][256]
   uint8_t* tcode = code_s + kCodeBytes;                                       // [2][256][16]
   float* red_m = reinterpret_cast<float*>(tcode + kTCodeBytes);              // [16][4]
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   stage_codebook(cw_s, kcb, rc, tid);
   stage_codes(t_begin, 0);
   cp_async_commit();
-  for (int i = tid; i < rc * kBinRow; i += kWThreads) bins[i] = 0.f;
+  for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) bins[i] = 0.f;
   if (tid < kWHeads) {
     mref_s[tid] = -INFINITY;
     l_s[tid] = 0.f;
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     }
     __syncthreads();
     if (fac_s[0] != 1.f || fac_s[1] != 1.f || fac_s[2] != 1.f || fac_s[3] != 1.f) {
-      for (int i = tid; i < rc * kBinRow; i += kWThreads) bins[i] *= fac_s[i & 3];
+      for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) bins[i] *= fac_s[i & 3];
       __syncthreads();
     }
     const float m = mref_s[hh];
@@ -303,22 +305,24 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     ls += __shfl_xor_sync(0xffffffffu, ls, 16);
     if (lane < kWHeads) red_l[warp * kWHeads + lane] = ls;
     // value reorder: the weight goes to the bin of the token's value code, per own round
-    if (wA > 0.f) {
-      const uint4 v4 = *reinterpret_cast<const uint4*>(tcode + (kWTile + tA) * 16);
-      const uint32_t vcw[4] = {v4.x, v4.y, v4.z, v4.w};
+    // token slot j of the warp starts at round j (mod rc), so each atomic instruction's 8
+    // tokens bin 8 different rounds
+    const int r_first = (lane >> 2) % rc;
+    auto bin_token = [&](int tt, float wt) {
+      const uint4 v4 = *reinterpret_cast<const uint4*>(tcode + (kWTile + tt) * 16);
+      int r = r_first;
 #pragma unroll
-      for (int r = 0; r < kRC; ++r)
-        if (r < rc)
-          atomicAdd(&bins[r * kBinRow + ((vcw[r >> 2] >> (8 * (r & 3))) & (kWideCodes - 1)) * kWHeads + hh], wA);
-    }
-    if (wB > 0.f) {
-      const uint4 v4 = *reinterpret_cast<const uint4*>(tcode + (kWTile + tB) * 16);
-      const uint32_t vcw[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-      for (int r = 0; r < kRC; ++r)
-        if (r < rc)
-          atomicAdd(&bins[r * kBinRow + ((vcw[r >> 2] >> (8 * (r & 3))) & (kWideCodes - 1)) * kWHeads + hh], wB);
-    }
+      for (int i = 0; i < kRC; ++i) {
+        if (i < rc) {
+          const uint32_t wd = r < 4 ? v4.x : (r < 8 ? v4.y : v4.z);
+          const int c = (wd >> (8 * (r & 3))) & (kWideCodes - 1);
+          atomicAdd(&bins[c * kBinStride + 4 * r + hh], wt);
+          r = (r + 1 == rc) ? 0 : r + 1;
+        }
+      }
+    };
+    if (wA > 0.f) bin_token(tA, wA);
+    if (wB > 0.f) bin_token(tB, wB);
   }
   __syncthreads();
   if (tid < kWHeads) {
@@ -338,10 +342,10 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   const int eh = (tid >> 6) & 3, ed = tid & 63, half = tid >> 8;
   float o = 0.f;
   for (int r = 0; r < rc; ++r) {
-    const float* br = bins + r * kBinRow + eh;
+    const float* br = bins + 4 * r + eh;
     const float* vr = cv + static_cast<size_t>(r) * kWideCodes * kWideVDims + ed;
 #pragma unroll 8
-    for (int c = half * 32; c < half * 32 + 32; ++c) o = fmaf(br[c * kWHeads], vr[c * kWideVDims], o);
+    for (int c = half * 32; c < half * 32 + 32; ++c) o = fmaf(br[c * kBinStride], vr[c * kWideVDims], o);
   }
   // the xchg buffer the last tile did not use: no peer reads it any more
   float* ored = xchg + (n_tiles & 1) * kWTile * kWHeads;   // [256] halves, then [256] slice
