@@ -52,3 +52,33 @@ def test_fuzz(i):
     out, lse = run_gpu(d, form=c["form"], n_splits=c["splits"])
     ref_out, ref_lse = run_oracle(d)
     assert_close(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("i", range(30))
+def test_fuzz_encode_append(i):
+    """The write side on random shapes: codes bit-exact with the oracle's, nothing else
+    written."""
+    import compressed_attention_cvq_b200 as cvq
+    from oracle import encode as E
+
+    rng = np.random.default_rng(3000 + i)
+    wide = rng.random() < 0.4
+    R = int(rng.integers(1, 23)) if wide else int(rng.integers(1, 3))
+    B, Hkv = int(rng.integers(1, 5)), int(rng.integers(1, 4))
+    T = 16 * int(rng.integers(1, 6)) if wide else int(rng.integers(1, 80))
+    d = workloads.small(batch=B, n_q_heads=4 * Hkv, n_kv_heads=Hkv, t_cap=T, R=R, seed=4000 + i,
+                        cb_std=math.sqrt(1.0 / R), group_dim=64 if wide else 8)
+    keys = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    vals = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    pos = rng.integers(-2, T + 2, size=B).astype(np.int32)
+    kc = np.full(d["key_codes"].shape, 0x5A, np.uint8)
+    vc = np.full(d["val_codes"].shape, 0x5A, np.uint8)
+    dk, dv = torch.from_numpy(kc.copy()).cuda(), torch.from_numpy(vc.copy()).cuda()
+    shape = cvq.make_shape(B, 4 * Hkv, Hkv, R, T, d["rope_base"], 128, 64 if wide else 8)
+    cvq.encode_append(shape, torch.from_numpy(keys).cuda(), torch.from_numpy(vals).cuda(),
+                      torch.from_numpy(d["key_cb"]).cuda(), torch.from_numpy(d["val_cb"]).cuda(),
+                      torch.from_numpy(pos).cuda(), dk, dv)
+    torch.cuda.synchronize()
+    E.encode_append(keys, vals, d["key_cb"], d["val_cb"], pos, kc, vc,
+                    codes_layout="planar" if wide else "token")
+    assert np.array_equal(dk.cpu().numpy(), kc) and np.array_equal(dv.cpu().numpy(), vc)
