@@ -82,3 +82,26 @@ def test_fuzz_encode_append(i):
     E.encode_append(keys, vals, d["key_cb"], d["val_cb"], pos, kc, vc,
                     codes_layout="planar" if wide else "token")
     assert np.array_equal(dk.cpu().numpy(), kc) and np.array_equal(dv.cpu().numpy(), vc)
+
+
+@pytest.mark.parametrize("i", range(12))
+def test_fuzz_larger(i):
+    """Fewer, larger random cases: several tiles per split, up to 8 KV heads, up to 200
+    splits (the fused merge walks many partial states)."""
+    rng = np.random.default_rng(5000 + i)
+    wide = rng.random() < 0.3
+    group = 4 if wide else int(rng.choice([1, 2, 4, 8]))
+    R = int(rng.integers(1, 23)) if wide else (1 if group == 8 else int(rng.integers(1, 3)))
+    T = 16 * int(rng.integers(64, 320)) if wide else int(rng.integers(1000, 5000))
+    B, Hkv = int(rng.integers(1, 4)), int(rng.integers(1, 9))
+    lens = rng.integers(0, T + 1, size=B).astype(np.int32)
+    lens[0] = T
+    splits = int(rng.integers(1, 201))
+    d = workloads.small(batch=B, n_q_heads=group * Hkv, n_kv_heads=Hkv, t_cap=T, R=R,
+                        q_dtype="bf16" if rng.random() < 0.5 else "f32", seq_lens=lens,
+                        seed=6000 + i, cb_std=math.sqrt(1.0 / R), group_dim=64 if wide else 8)
+    out, lse = run_gpu(d, form="gqa", n_splits=splits)
+    heads = [(b, h) for b in range(B) for h in rng.choice(group * Hkv, size=min(6, group * Hkv),
+                                                           replace=False)]
+    ref_out, ref_lse = run_oracle(d, heads=heads)
+    assert_close(out, lse, ref_out, ref_lse, heads=heads)
