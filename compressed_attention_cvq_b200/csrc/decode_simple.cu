@@ -183,18 +183,62 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
       a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = m_run[tid] * kLn2;
     }
   }
-  // epilogue: o[hh][8G + d] = sum_{r, c} bins[hh][G][r][c] * val_cb[G][r][c][d]
-  const float* vcb = a.val_cb + static_cast<size_t>(h) * a.val_cb_stride;
-  for (int i = tid; i < NG * kHeadDim; i += kSimpleThreads) {
-    const int hh = i / kHeadDim, dim = i % kHeadDim;
-    const int G = dim / kVDims, d = dim % kVDims;
-    const float* bh = bins + (hh * kGroups + G) * R * kCodes;
-    float acc = 0.f;
-#pragma unroll 16
-    for (int rc = 0; rc < R * kCodes; ++rc) {
-      acc = fmaf(bh[rc], __ldg(vcb + (static_cast<size_t>(G) * R * kCodes + rc) * kVDims + d), acc);
+  // epilogue: o[hh][8G + d] = sum_{r, c} bins[hh][G][r][c] * val_cb[G][r][c][d].
+  // Thread = (group G, code lane ch): it sums the codes ch, ch + 16, ... of its group over
+  // all 8 dims of the group (two 16-byte loads per code, many in flight), then the 16 code
+  // lanes of a half-warp reduce-scatter their 8 sums so that each dim ends on one lane.
+  {
+    static_assert(kGroups * 16 == kSimpleThreads, "one thread per (group, code lane)");
+    constexpr int kSteps = R * kCodes / 16;
+    const int G = tid >> 4, ch = tid & 15;
+    const float4* vcb = reinterpret_cast<const float4*>(a.val_cb + static_cast<size_t>(h) * a.val_cb_stride) +
+                        static_cast<size_t>(G) * R * kCodes * 2;
+    float acc[NG][8];
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+#pragma unroll
+      for (int d = 0; d < 8; ++d) acc[hh][d] = 0.f;
     }
-    a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + dim] = acc;
+    // odd groups start one step later: the two half-warps then read opposite bank halves
+    const int k0 = G & 1;
+#pragma unroll 8
+    for (int k = 0; k < kSteps; ++k) {
+      const int kk = (k + k0 == kSteps) ? 0 : k + k0;
+      const int rc = kk * 16 + ch;                      // r * 256 + c
+      const float4 v0 = __ldg(vcb + rc * 2), v1 = __ldg(vcb + rc * 2 + 1);
+#pragma unroll
+      for (int hh = 0; hh < NG; ++hh) {
+        const float w = bins[(hh * kGroups + G) * R * kCodes + rc];
+        acc[hh][0] = fmaf(w, v0.x, acc[hh][0]); acc[hh][1] = fmaf(w, v0.y, acc[hh][1]);
+        acc[hh][2] = fmaf(w, v0.z, acc[hh][2]); acc[hh][3] = fmaf(w, v0.w, acc[hh][3]);
+        acc[hh][4] = fmaf(w, v1.x, acc[hh][4]); acc[hh][5] = fmaf(w, v1.y, acc[hh][5]);
+        acc[hh][6] = fmaf(w, v1.z, acc[hh][6]); acc[hh][7] = fmaf(w, v1.w, acc[hh][7]);
+      }
+    }
+    const bool b3 = ch & 8, b2 = ch & 4, b1 = ch & 2;
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+      float* v = acc[hh];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {      // lanes differing in bit 3: keep dims 4 b3 + i
+        const float send = b3 ? v[i] : v[i + 4];
+        v[i] = (b3 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {      // bit 2: keep dims 4 b3 + 2 b2 + i
+        const float send = b2 ? v[i] : v[i + 2];
+        v[i] = (b2 ? v[i + 2] : v[i]) + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      {                                  // bit 1: keep dim 4 b3 + 2 b2 + b1
+        const float send = b1 ? v[0] : v[1];
+        v[0] = (b1 ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+      if ((ch & 1) == 0) {
+        const int dim = G * kVDims + (ch >> 1);         // ch >> 1 = 4 b3 + 2 b2 + b1
+        a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + dim] = v[0];
+      }
+    }
   }
   if constexpr (!TABLE) {
     if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
