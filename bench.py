@@ -501,6 +501,9 @@ def run_gpu(args):
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / n_e2e, dev)
+    fault = cvq.fault_status(clear=True)     # a bounded codebook-copy wait gave up: invalid run
+    if fault:
+        raise RuntimeError(f"device fault word {fault:#x} after the timed steps")
 
     result = None
     if rank == 0:
@@ -548,6 +551,7 @@ def run_gpu(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "smem_floor": smem_summary(w, total_tokens, dec_mean_ms, pk, args.form),
             "gpu_launches": args.steps * launches_per_step,
+            "device_faults": fault,
             "_layer0": layer0,
             "append": append_summary(w, enc_ms) if args.append else None,
             "clocks": clk.summary(),

@@ -9,6 +9,7 @@ The calls of the library, one-to-one with include/cvq.h:
   attend_fused(shape, q, key_cb, codes...)       -> (out, lse)   (cvq_attend)
   naive_dequant / naive_decode                   -> the comparison path
   encode_append(shape, keys, values, ...)        -> codes written (cvq_encode_append)
+  fault_status(clear)                            -> device fault bits (cvq_fault_status)
 
 plus attend(), which allocates the intermediate buffers with torch and runs the calls in
 order.  Tensors are torch CUDA tensors in the layouts documented in cvq.h; work is
@@ -27,7 +28,7 @@ from ._binding import CVQ_BF16, CVQ_F32, CvqError, cvq_shape, make_shape  # noqa
 __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa", "combine",
            "attend", "naive_dequant", "naive_decode", "encode_append", "split_tokens",
            "suggest_splits", "partials_alloc", "group_dim_of", "attend_fused", "workspace_alloc",
-           "CvqError"]
+           "fault_status", "CvqError"]
 
 
 def _ptr(t):
@@ -185,6 +186,16 @@ def attend_fused(shape, q, key_cb, key_codes, val_codes, seq_lens, val_cb, n_spl
                            _ptr(workspace), _ptr(out), _ptr(lse), _stream(stream))
     _b.check(st, "cvq_attend")
     return out, lse
+
+
+def fault_status(clear=False, device=None):
+    """The device fault word of the current (or given) CUDA device: 0, or CVQ_FAULT_* bits
+    set by a kernel whose bounded wait on a codebook copy gave up.  Synchronizes the device."""
+    flags = ctypes.c_uint32(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        st = _b.lib.cvq_fault_status(ctypes.byref(flags), 1 if clear else 0)
+    _b.check(st, "cvq_fault_status")
+    return int(flags.value)
 
 
 def combine(shape, n_splits, part_o, part_m, part_l, out=None, lse=None, stream=None):

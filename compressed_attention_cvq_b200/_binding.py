@@ -58,6 +58,7 @@ def _load():
         "cvq_encode_append": (I, [S, P, P, P, I64, P, I64, P, P, P, P]),
         "cvq_attend_workspace_bytes": (SZ, [S, I]),
         "cvq_attend": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P, P]),
+        "cvq_fault_status": (I, [ctypes.POINTER(ctypes.c_uint32), I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -82,7 +83,9 @@ EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partia
             "cvq_split_tokens", "cvq_suggest_splits", "cvq_qtable", "cvq_decode_attn",
             "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static",
             "cvq_naive_cache_bytes", "cvq_naive_dequant", "cvq_naive_decode",
-            "cvq_encode_append", "cvq_attend_workspace_bytes", "cvq_attend"]
+            "cvq_encode_append", "cvq_attend_workspace_bytes", "cvq_attend",
+            "cvq_fault_status"]
+CVQ_FAULT_COPY_TIMEOUT = 1
 
 
 def status_str(st: int) -> str:

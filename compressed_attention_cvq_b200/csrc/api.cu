@@ -1,6 +1,6 @@
 // libcvq C ABI: argument validation on the host, then kernel launches.  Nothing is
-// allocated and no state is kept; every error is returned as a cvq_status before any
-// launch.
+// allocated; the only state is the device fault word (device_state.cu).  Every argument
+// error is returned as a cvq_status before any launch.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -133,6 +133,12 @@ cvq_status decode_gqa_impl(const cvq_shape* s, const void* q, int q_dtype, const
   a.counters = counters;
   a.out = out;
   a.lse = lse;
+  if (fault_word_address(&a.fault) != cudaSuccess) return CVQ_ERR_CUDA;
+  if (!is_wide(s) && s->n_q_heads / s->n_kv_heads == 4) {   // the kernel that stages by TMA maps
+    if (encode_codebook_map(&a.key_map, key_cb, key_cb_head_stride, s->n_kv_heads, s->R) != cudaSuccess ||
+        encode_codebook_map(&a.val_map, val_cb, val_cb_head_stride, s->n_kv_heads, s->R) != cudaSuccess)
+      return CVQ_ERR_CUDA;
+  }
   if (is_wide(s)) return from_cuda(launch_decode_wide(*s, a, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
 }

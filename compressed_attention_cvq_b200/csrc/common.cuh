@@ -2,6 +2,7 @@
 // fixed-point turns, and small device helpers.
 #pragma once
 
+#include <cuda.h>            // CUtensorMap (the type only; the encoder is reached at run time)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -103,7 +104,78 @@ struct DecodeArgs {
   int* counters;
   float* out;
   float* lse;
+  // 4-query-head kernel only: tiled TMA maps of the key and value codebooks (see
+  // encode_codebook_map), read from the kernel parameter space
+  CUtensorMap key_map;
+  CUtensorMap val_map;
+  // device fault word of the library (kFault* bits), set when a bounded wait gives up
+  unsigned int* fault;
 };
+
+// ---- bits of the device fault word (cvq_fault_status) ----
+constexpr unsigned int kFaultCopyTimeout = CVQ_FAULT_COPY_TIMEOUT;   // a TMA copy did not land in time
+
+constexpr int kCodeBoxRows = 32;   // codes per TMA box of the codebook maps
+
+// ---- mbarrier + TMA (bulk copy engine) helpers ----
+// try_wait rounds before a wait gives up; each round suspends the thread for at most about
+// the hint below (ns), so the limit is a few seconds
+constexpr int kMbarTries = 1 << 22;
+constexpr unsigned int kMbarSuspendNs = 1000u;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// arrive once and add `bytes` to the transaction count the current phase waits for
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned int bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Wait (bounded) for the completion of the phase with the given parity; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned int parity) {
+  const uint32_t addr = smem_u32(bar);
+  unsigned long long t0 = 0;
+  for (int i = 0;; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    unsigned long long now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    if (i == 0) t0 = now;
+    else if (now - t0 > 2000000000ull) return false;
+  }
+}
+// order this thread's earlier generic-proxy shared-memory accesses before later TMA writes
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 4-d tiled tensor copy, global -> this CTA's shared memory, completing on `bar`
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+// contiguous bulk copy, global -> this CTA's shared memory (both addresses 16-byte aligned,
+// bytes a multiple of 16), completing on `bar`
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned int bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // The split merge of cvq_combine, fused into the end of a decode kernel.  Every CTA of a
 // work unit (sequence b, grid row `unit` = blockIdx.y) calls this with all its threads
@@ -206,6 +278,15 @@ cudaError_t launch_naive_decode(const cvq_shape& s, const void* q, int q_dtype, 
                                 cudaStream_t stream);
 // 64-scalar groups, 4 query heads per KV head (decode_wide.cu)
 cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+
+// Host side of the TMA staging and the fault word (device_state.cu).
+// Tiled map of one codebook tensor (key or value, narrow layout: per head [16 groups][R][256
+// codes][8 floats], heads head_stride floats apart, 0 = one codebook for all heads) whose
+// box is 8 groups x kCodeBoxRows codes of one round, landing as [code][local group][8
+// floats] (16-byte chunk (code * 8 + local group) * 2 + half).
+cudaError_t encode_codebook_map(CUtensorMap* map, const float* base, long long head_stride,
+                                int n_heads, int R);
+cudaError_t fault_word_address(unsigned int** out);
 // the write side: greedy residual encoding of one new key / value per (sequence, KV head)
 cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const float* values,
                                  const float* key_cb, long long key_stride, const float* val_cb,

@@ -20,8 +20,10 @@
 //   6. epilogue: o = bins x value codebook for the CTA's 64 output dims.
 //
 // Shared-memory layouts, chosen for conflict-free access (32 banks x 4 bytes):
-//   key / value codewords: 16-byte chunk ((r*256 + c)*2 + half)*8 + G_local, so the 8
-//     lanes of a quarter-warp (one token, groups 0..7) hit 8 different bank groups;
+//   key / value codewords: [r][c][G_local][8 floats], staged by TMA (8 tiled copies of
+//     32 codes per round, 32-byte rows); the lanes of groups 0-3 read the lower 16-byte
+//     half of their codeword first and those of groups 4-7 the upper half, so the 8 lanes
+//     of a quarter-warp (one token, groups 0..7) hit 8 different bank groups;
 //   bins: float ((r*256 + c)*4 + head)*8 + G_local; at every atomic step the 32 lanes
 //     of a warp (4 tokens x 4 heads x 2 group halves, each token on a rotated group)
 //     touch 32 different banks and never the same address.
@@ -60,20 +62,31 @@ struct Cfg {
   static constexpr int kCodeBytes = 2 * kTile * R * 16;               // 2 buffers x (key 8 B + val 8 B) x R
   static constexpr size_t kSmem = sizeof(float4) * kCodeChunks +
                                   sizeof(float) * (kBins + kXchg + kWarps * kHeads + 2 * kHeads) +
-                                  kCodeBytes;
+                                  kCodeBytes + 16;   // + the TMA mbarrier
   static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
 };
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
 __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
   const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// One CTA's half of a codebook (local groups 8 rank .. 8 rank + 7, every round and code)
+// into the chunk layout of cw_s, by 8 R tiled TMA copies of 32 codes each, issued by lanes
+// 0 .. 8R-1 of one warp after lane 0 set the transaction count.  Called by a whole warp.
+template <int R>
+__device__ __forceinline__ void stage_codebook_tma(float4* cw_s, const CUtensorMap* map, int rank, int head,
+                                                   uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) mbar_expect_tx(bar, static_cast<unsigned>(sizeof(float4)) * R * kCodes * 2 * kLocalGroups);
+  __syncwarp();
+  if (lane < 8 * R) {
+    const int rc = lane * kCodeBoxRows;                 // round * 256 + first code
+    tma_load_4d(cw_s + rc * kLocalGroups * 2, map, 0, rank * kLocalGroups, rc, head, bar);
+  }
+}
 
 __device__ __forceinline__ void cluster_arrive_release() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -88,16 +101,17 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
 
 template <int R>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cfg<R>::kMinBlocks)
-    decode_gqa4_kernel(const DecodeArgs a) {
+    decode_gqa4_kernel(const __grid_constant__ DecodeArgs a) {
   using C = Cfg<R>;
-  extern __shared__ float4 smem4[];
-  float4* cw_s = smem4;                                               // [R][256][2][8] chunks
+  extern __shared__ __align__(128) float4 smem4[];
+  float4* cw_s = smem4;                                               // [R][256][8][2] chunks
   float* bins = reinterpret_cast<float*>(smem4 + C::kCodeChunks);     // [R][256][4][8]
   float* xchg = bins + C::kBins;                                      // [2][kTile][4]
   float* red = xchg + C::kXchg;                                       // [kWarps][4]
   float* fh = red + C::kWarps * kHeads;                               // [4] tile max / factors
   float* mtile = fh + kHeads;                                         // [4]
   uint8_t* code_s = reinterpret_cast<uint8_t*>(mtile + kHeads);       // [2][kTile][R][key 8 | val 8]
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(code_s + C::kCodeBytes);   // codebook copies
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());           // which half of the groups
@@ -108,6 +122,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   const int warp = tid >> 5, lane = tid & 31;
   const int tau = lane >> 3;               // token slot within the warp (0..3)
   const int k = lane & 7;                  // local group of the key side
+  const int fk = k >> 2;                   // which codeword half this lane reads first
   const int hk = k & 3;                    // head whose score / weights this lane keeps
   const int gh = k >> 2;                   // which 4 local groups this lane bins
   const int sigma = warp * 4 + tau;        // token slot within the step
@@ -148,12 +163,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     cp_async_commit();
   };
 
-  // ---- prologue: key codewords of this CTA's groups, first tile's codes (async) ----
-  const float4* kcb = reinterpret_cast<const float4*>(a.key_tab + static_cast<size_t>(h) * a.key_tab_stride);
-  for (int i = tid; i < C::kCodeChunks; i += C::kThreads) {
-    const int gl = i & 7, half = (i >> 3) & 1, c = (i >> 4) & 255, r = i >> 12;
-    const int G = rank * kLocalGroups + gl;
-    cp_async16(cw_s + i, kcb + ((static_cast<size_t>(G) * R + r) * kCodes + c) * 2 + half);
+  // ---- prologue: key codewords of this CTA's groups by TMA (tiled copies of groups
+  // 8 rank .. 8 rank + 7, straight into the layout above), the first tile's codes by
+  // cp.async ----
+  if (warp == 0) {
+    if (lane == 0) mbar_init(tma_bar, 1);
+    stage_codebook_tma<R>(cw_s, &a.key_map, rank, a.key_tab_stride == 0 ? 0 : h, tma_bar);
   }
   stage_codes(t_begin, 0);
   for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] = 0.f;
@@ -162,6 +177,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   // units.  Slot j holds head (k ^ j) & 3: with this lane-dependent order the butterfly
   // that sums the partials over the token's 8 lanes needs no selects, and leaves head
   // k & 3 in lanes k and k ^ 4.
+  // Lanes k = 4..7 read the upper half (pairs 2, 3) of their codeword first, so their
+  // slots 0..3 hold pairs 2, 3, 0, 1 of the group (fk = 1); lanes 0..3 keep pairs 0..3.
   const float qscale = kLog2e * 0.08838834764831845f;
   const int G = rank * kLocalGroups + k;
   float2 qv[kHeads][4];
@@ -171,15 +188,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     const size_t qb = (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim + 8 * G;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      qv[j][p] = make_float2(load_q(a.q, a.q_dtype, qb + 2 * p) * qscale,
-                             load_q(a.q, a.q_dtype, qb + 2 * p + 1) * qscale);
+      const int pp = p ^ (2 * fk);                     // slot p holds pair 4 G + pp
+      qv[j][p] = make_float2(load_q(a.q, a.q_dtype, qb + 2 * pp) * qscale,
+                             load_q(a.q, a.q_dtype, qb + 2 * pp + 1) * qscale);
     }
   }
   float2 ph[4], adv[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    ph[p] = phase_at(a.phase.F[4 * G + p], t_begin + sigma);
-    adv[p] = phase_at(a.phase.F[4 * G + p], C::kSlots);
+    const int pp = p ^ (2 * fk);
+    ph[p] = phase_at(a.phase.F[4 * G + pp], t_begin + sigma);
+    adv[p] = phase_at(a.phase.F[4 * G + pp], C::kSlots);
   }
   float* peer_xchg = cluster.map_shared_rank(xchg, rank ^ 1);
 
@@ -187,7 +206,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   float l_acc = 0.f;            // this lane's share of sum_t w for head hk
 
   cp_async_wait_all();
-  cluster.sync();               // codewords, bins and the first codes ready in both CTAs
+  cluster.sync();               // bins and the first codes ready in both CTAs
+  // the codewords (phase 0 of the barrier); a copy that never lands is reported in the
+  // fault word and the kernel runs on, so that every CTA still meets every barrier
+  if (!mbar_wait(tma_bar, 0) && tid == 0) atomicOr(a.fault, kFaultCopyTimeout);
 
   // per-lane float offsets into the bins: step i of a token's atomics adds to local group
   // 4 gh + ((i + tau) & 3) of head hk
@@ -247,8 +269,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int c = cb[(tt * R + r) * 16 + k];
-        const float4* src = cw_s + (r * kCodes + c) * (2 * kLocalGroups) + k;
-        const float4 lo = src[0], hi = src[kLocalGroups];
+        // chunk fk first: lanes 0-3 and 4-7 of a token then hit 8 distinct bank quads;
+        // lo holds the lane's slots 0, 1 and hi its slots 2, 3 (pairs 2 fk, ... see qv)
+        const float4* src = cw_s + ((r * kCodes + c) * kLocalGroups + k) * 2;
+        const float4 lo = src[fk], hi = src[fk ^ 1];
         if (r == 0) {
           kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
           kw[2] = make_float2(hi.x, hi.y); kw[3] = make_float2(hi.z, hi.w);
@@ -363,26 +387,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 
   // ---- epilogue: o[head][8 G + d] = sum_{r,c} bins[r][c][head][G] * val_cb[G][r][c][d] ----
   // value codewords of this CTA's groups replace the key codewords, same chunk layout
-  const float4* vcb = reinterpret_cast<const float4*>(a.val_cb + static_cast<size_t>(h) * a.val_cb_stride);
-  for (int i = tid; i < C::kCodeChunks; i += C::kThreads) {
-    const int gl = i & 7, half = (i >> 3) & 1, c = (i >> 4) & 255, r = i >> 12;
-    const int Gv = rank * kLocalGroups + gl;
-    cp_async16(cw_s + i, vcb + ((static_cast<size_t>(Gv) * R + r) * kCodes + c) * 2 + half);
+  // (every read of the key codewords happened before the barrier above; the fence orders
+  // them before the TMA writes)
+  if (warp == 0) {
+    fence_proxy_async_smem();
+    stage_codebook_tma<R>(cw_s, &a.val_map, rank, a.val_cb_stride == 0 ? 0 : h, tma_bar);
   }
-  cp_async_commit();
-  cp_async_wait_all();
-  __syncthreads();
+  if (!mbar_wait(tma_bar, 1) && tid == 0) atomicOr(a.fault, kFaultCopyTimeout);
   {
     // warp = slice of codes, lane = (head, local group): bins reads are 32 consecutive
-    // floats, codeword reads 8 distinct chunks in 8 bank groups
-    const int gl = lane & 7, hh = lane >> 3;
+    // floats; codeword reads take chunk fv first (dims 4 fv .. 4 fv + 3 in acc[0..3]) so
+    // that the 8 groups hit 8 distinct bank quads
+    const int gl = lane & 7, hh = lane >> 3, fv = gl >> 2;
     constexpr int kPerSlice = R * kCodes / C::kWarps;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int ci = 0; ci < kPerSlice; ++ci) {
       const int rc = warp * kPerSlice + ci;            // r * 256 + c
       const float wgt = bins[(rc * kHeads + hh) * kLocalGroups + gl];
-      const float4 v0 = cw_s[(rc * 2) * kLocalGroups + gl];
-      const float4 v1 = cw_s[(rc * 2 + 1) * kLocalGroups + gl];
+      const float4 v0 = cw_s[(rc * kLocalGroups + gl) * 2 + fv];
+      const float4 v1 = cw_s[(rc * kLocalGroups + gl) * 2 + (fv ^ 1)];
       acc[0] = fmaf(wgt, v0.x, acc[0]); acc[1] = fmaf(wgt, v0.y, acc[1]);
       acc[2] = fmaf(wgt, v0.z, acc[2]); acc[3] = fmaf(wgt, v0.w, acc[3]);
       acc[4] = fmaf(wgt, v1.x, acc[4]); acc[5] = fmaf(wgt, v1.y, acc[5]);
@@ -391,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     __syncthreads();                                   // bins no longer read: reuse them
     float* part_s = bins;                              // [kWarps][32 lanes][8]
 #pragma unroll
-    for (int d = 0; d < 8; ++d) part_s[(warp * 32 + lane) * 8 + d] = acc[d];
+    for (int d = 0; d < 8; ++d) part_s[(warp * 32 + lane) * 8 + d] = acc[d ^ (4 * fv)];
     __syncthreads();
     for (int o = tid; o < kHeads * kLocalGroups * 8; o += C::kThreads) {
       const int d = o & 7, ln = o >> 3;                // ln = head * 8 + local group

@@ -62,6 +62,11 @@ constexpr size_t kRedBytes = sizeof(float) * (2 * kWWarps * kWHeads + 4 * kWHead
 constexpr size_t kWSmem = kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kTCodeBytes + kRedBytes;
 static_assert(kWSteps * kWSlots == kWTile, "tile must be a whole number of steps");
 static_assert(kWSmem <= 227 * 1024, "shared memory per CTA");
+// the reduction region holds red_m, red_l, mref_s, l_s, fac_s and, in its last 16 bytes, the
+// 8-byte mbarrier of the codebook copies
+static_assert(kRedBytes >= sizeof(float) * (2 * kWWarps * kWHeads + 3 * kWHeads) + 8, "mbarrier room");
+static_assert((kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kTCodeBytes +
+               sizeof(float) * (2 * kWWarps * kWHeads + 3 * kWHeads)) % 8 == 0, "mbarrier alignment");
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -78,15 +83,19 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
   return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
 }
 
-// Copy rc rounds x 64 codewords of one group (a contiguous run of rc * 4096 floats).
-__device__ __forceinline__ void stage_codebook(float4* dst, const float* src, int rc, int tid) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-  const int n = rc * kWideCodes * kWChunks;
-  for (int i = tid; i < n; i += kWThreads) cp_async16(dst + i, s4 + i);
+// Copy rc rounds x 64 codewords of one group (a contiguous run of rc * 4096 floats) with
+// one TMA bulk copy per round, issued by lanes 0 .. rc-1 of warp 0 after lane 0 set the
+// transaction count.
+__device__ __forceinline__ void stage_codebook(float4* dst, const float* src, int rc, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  constexpr unsigned kRound = static_cast<unsigned>(sizeof(float4)) * kWideCodes * kWChunks;
+  if (lane == 0) mbar_expect_tx(bar, kRound * rc);
+  __syncwarp();
+  if (lane < rc) bulk_load(dst + lane * kWideCodes * kWChunks, src + lane * kWideCodes * 4 * kWChunks, kRound, bar);
 }
 
 __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeArgs a, int R) {
-  extern __shared__ float4 smem4[];
+  extern __shared__ __align__(128) float4 smem4[];
   float4* cw_s = smem4;                                                       // codewords
   float* bins = reinterpret_cast<float*>(smem4 + kRC * kWideCodes * kWChunks);
   float* xchg = bins + kWideCodes * kBinStride;                               // [2][256][4]
@@ -97,6 +106,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   float* mref_s = red_l + kWWarps * kWHeads;                                  // [4]
   float* l_s = mref_s + kWHeads;                                              // [4]
   float* fac_s = l_s + kWHeads;                                               // [4]
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(fac_s + kWHeads);           // codebook copies
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -152,7 +162,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 
   const float* kcb = a.key_tab + h * a.key_tab_stride +
                      (static_cast<size_t>(G) * R + r0) * kWideCodes * 2 * kWidePairs;
-  stage_codebook(cw_s, kcb, rc, tid);
+  if (tid == 0) mbar_init(tma_bar, 1);
+  if (warp == 0) stage_codebook(cw_s, kcb, rc, tma_bar);
   stage_codes(t_begin, 0);
   cp_async_commit();
   for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) bins[i] = 0.f;
@@ -195,7 +206,10 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     const int t_tile = t_begin + it * kWTile;
     const int buf = it & 1;
     cp_async_wait_all();
-    __syncthreads();                          // codes of this tile (and the codebook) landed
+    __syncthreads();                          // codes of this tile landed
+    // the key codewords (phase 0 of the barrier); a copy that never lands is reported in
+    // the fault word and the kernel runs on, so that every CTA still meets every barrier
+    if (it == 0 && !mbar_wait(tma_bar, 0) && tid == 0) atomicOr(a.fault, kFaultCopyTimeout);
     if (it + 1 < n_tiles) stage_codes(t_tile + kWTile, buf ^ 1);
     cp_async_commit();
     // token-major copy of this tile's codes: 16 bytes per (key | value, token), byte r =
@@ -334,10 +348,13 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   // ---- epilogue: o = bins x value codewords of the own rounds ----
   const float* vcb = a.val_cb + h * a.val_cb_stride +
                      (static_cast<size_t>(G) * R + r0) * kWideCodes * kWideVDims;
-  stage_codebook(cw_s, vcb, rc, tid);
-  cp_async_commit();
-  cp_async_wait_all();
-  __syncthreads();
+  // (every read of the key codewords happened before the barrier above; the fence orders
+  // them before the TMA writes)
+  if (warp == 0) {
+    fence_proxy_async_smem();
+    stage_codebook(cw_s, vcb, rc, tma_bar);
+  }
+  if (!mbar_wait(tma_bar, 1) && tid == 0) atomicOr(a.fault, kFaultCopyTimeout);
   const float* cv = reinterpret_cast<const float*>(cw_s);
   const int eh = (tid >> 6) & 3, ed = tid & 63, half = tid >> 8;
   float o = 0.f;

@@ -31,13 +31,17 @@
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers, owned by the caller, row-major, and
- *     16-byte aligned.  The library allocates nothing and keeps no state between calls.
+ *     16-byte aligned.  The library allocates nothing; the only state it keeps between
+ *     calls is one device fault word per GPU (cvq_fault_status).
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL = legacy
  *     default stream).  A status of CVQ_OK means the launch was accepted.
  *   - Argument errors are detected on the host before any launch and returned as a
  *     status; nothing is launched then.  Launch failures map to CVQ_ERR_CUDA.  No call
  *     throws across the ABI.
  *   - seq_lens[b] is read on the device and clamped to [0, t_cap].
+ *   - The first GQA decode call on a device (cvq_decode_attn_gqa, cvq_attend,
+ *     cvq_attend_static) looks up the device fault word's address with that device
+ *     current; make it before any stream capture.
  */
 #ifndef CVQ_H
 #define CVQ_H
@@ -293,6 +297,22 @@ CVQ_API cvq_status cvq_attend_static(const cvq_shape* shape, const void* q, int 
                                      const int32_t* seq_lens, const float* val_cb,
                                      int64_t val_cb_head_stride, int n_splits, float* out,
                                      float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_fault_status -- the device fault word of the current device.  The decode kernels
+ * that stage codebooks with the TMA engine (cvq_decode_attn_gqa / cvq_attend /
+ * cvq_attend_static with 4 query heads per KV head, and every g = 64 decode) wait for
+ * those copies with a bounded wait; if a wait gives up, the kernel sets a bit here and
+ * runs to completion (its outputs are then invalid) instead of hanging the GPU.
+ *   Bits: CVQ_FAULT_COPY_TIMEOUT = a codebook copy did not land within the wait limit.
+ *   flags (host): receives the word.  clear != 0 resets it to 0 afterwards.
+ *   Synchronous: waits for the device (cudaMemcpy).  The first call on a device looks up
+ *   the word's address (cudaGetSymbolAddress), as the first decode call does; make that
+ *   first call before any stream capture.
+ *   Errors: CVQ_ERR_NULL (flags NULL), CVQ_ERR_CUDA.
+ * ------------------------------------------------------------------------------- */
+#define CVQ_FAULT_COPY_TIMEOUT 1u
+CVQ_API cvq_status cvq_fault_status(uint32_t* flags, int clear);
 
 #ifdef __cplusplus
 }
