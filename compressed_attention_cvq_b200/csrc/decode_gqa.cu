@@ -218,6 +218,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   for (int i = 0; i < 4; ++i) bin_off[i] = hk * kLocalGroups + 4 * gh + ((i + tau) & 3);
 
   const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
+  // With one CTA per SM (R = 2) nothing hides this CTA's tail, so the value codebook copy
+  // starts as soon as the last key gather is done; with two per SM the other CTA covers it
+  // and the early copy only costs registers (measured: Zipf batch 254 -> 248 us, 32K R = 2
+  // 81.8 -> 80.9 us, 128K R = 1 +0.5-1 us).
+  constexpr bool kEarlyValueCopy = C::kMinBlocks == 1;
 
   // Software pipeline over tiles.  Iteration t: key side of tile t -> arrive on the
   // cluster barrier -> bin atomics of tile t-1 (weights and value codes kept in
@@ -255,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   };
 
   // one tile: FULL = every token of the tile is inside the split (no per-token checks)
-  auto run_tile = [&](const int t_tile, const int buf, auto full_tag) {
+  auto run_tile = [&](const int t_tile, const int buf, auto full_tag, const bool last) {
     constexpr bool FULL = decltype(full_tag)::value;
     const uint8_t* cb = code_s + static_cast<size_t>(buf) * kTile * R * 16;
     float* xb = xchg + buf * (kTile * kHeads);
@@ -305,6 +310,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     cluster_arrive_release();
     bin_atomics();                      // previous tile, while the exchange completes
     cluster_wait_acquire();             // the peer's partials of this tile are in xb
+    if (kEarlyValueCopy && last && warp == 0) {
+      // every thread of the CTA is past its last key gather: bring in the value codewords
+      // over the key codewords now, behind this tile's softmax, bins and the l reduction
+      // (the fence orders the gathers before the TMA writes)
+      fence_proxy_async_smem();
+      stage_codebook_tma<R>(cw_s, &a.val_map, rank, a.val_cb_stride == 0 ? 0 : h, tma_bar);
+    }
 
     // full scores (the same order of addition in both CTAs -> identical values)
     float s[C::kSteps];
@@ -363,9 +375,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     }
     if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
     if (t_tile + kTile <= t_end) {
-      run_tile(t_tile, buf, std::integral_constant<bool, true>());
+      run_tile(t_tile, buf, std::integral_constant<bool, true>(), tile + 1 == n_tiles);
     } else {
-      run_tile(t_tile, buf, std::integral_constant<bool, false>());
+      run_tile(t_tile, buf, std::integral_constant<bool, false>(), tile + 1 == n_tiles);
     }
   }
   bin_atomics();                // the last tile
@@ -386,10 +398,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   }
 
   // ---- epilogue: o[head][8 G + d] = sum_{r,c} bins[r][c][head][G] * val_cb[G][r][c][d] ----
-  // value codewords of this CTA's groups replace the key codewords, same chunk layout
-  // (every read of the key codewords happened before the barrier above; the fence orders
-  // them before the TMA writes)
-  if (warp == 0) {
+  // the value codewords of this CTA's groups, over the key codewords in the same layout
+  // (copied since the last tile's cluster barrier if kEarlyValueCopy; else now: every read
+  // of the key codewords happened before the barrier above, the fence orders them before
+  // the TMA writes)
+  if (!kEarlyValueCopy && warp == 0) {
     fence_proxy_async_smem();
     stage_codebook_tma<R>(cw_s, &a.val_map, rank, a.val_cb_stride == 0 ? 0 : h, tma_bar);
   }

@@ -22,8 +22,9 @@
 // the round slices of one group add their outputs through distributed shared memory.
 //
 // Layouts in shared memory (32 banks x 4 bytes):
-//   key / value codewords: [rc][64 codes][16 chunks of 16 bytes]; lane k of a token reads
-//     chunks k and 8 + k, so the 8 lanes of a quarter-warp read 128 contiguous bytes;
+//   key / value codewords: [rc][64 codes][16 chunks of 16 bytes] -- the global layout of
+//     the group's rounds, so each round arrives by one TMA bulk copy; lane k of a token
+//     reads chunks k and 8 + k, so the 8 lanes of a quarter-warp read 128 contiguous bytes;
 //   bins: float c * 64 + 4 r + head; a warp's 8 tokens bin 8 different rounds at each
 //     atomic step (the token's slot in the warp rotates its round order), so the 32 lanes
 //     of an atomic hit 32 different banks whatever the codes;
@@ -162,6 +163,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 
   const float* kcb = a.key_tab + h * a.key_tab_stride +
                      (static_cast<size_t>(G) * R + r0) * kWideCodes * 2 * kWidePairs;
+  const float* vcb = a.val_cb + h * a.val_cb_stride +
+                     (static_cast<size_t>(G) * R + r0) * kWideCodes * kWideVDims;
   if (tid == 0) mbar_init(tma_bar, 1);
   if (warp == 0) stage_codebook(cw_s, kcb, rc, tma_bar);
   stage_codes(t_begin, 0);
@@ -346,8 +349,6 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   }
 
   // ---- epilogue: o = bins x value codewords of the own rounds ----
-  const float* vcb = a.val_cb + h * a.val_cb_stride +
-                     (static_cast<size_t>(G) * R + r0) * kWideCodes * kWideVDims;
   // (every read of the key codewords happened before the barrier above; the fence orders
   // them before the TMA writes)
   if (warp == 0) {
