@@ -171,7 +171,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     stage_codebook_tma<R>(cw_s, &a.key_map, rank, a.key_tab_stride == 0 ? 0 : h, tma_bar);
   }
   stage_codes(t_begin, 0);
-  for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] = 0.f;
+  for (int i = tid; i < C::kBins / 4; i += C::kThreads)
+    reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 
   // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2
   // units.  Slot j holds head (k ^ j) & 3: with this lane-dependent order the butterfly

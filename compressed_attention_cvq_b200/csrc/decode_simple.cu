@@ -67,7 +67,8 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
     }
     qs[hh][d] = v;
   }
-  for (int i = tid; i < NG * kGroups * R * kCodes; i += kSimpleThreads) bins[i] = 0.f;
+  for (int i = tid; i < NG * kGroups * R * kCodes / 4; i += kSimpleThreads)
+    reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 
   const float* tab = TABLE ? a.key_tab + (static_cast<size_t>(b) * a.n_q_heads + head) * a.key_tab_stride
                            : a.key_tab + static_cast<size_t>(h) * a.key_tab_stride;

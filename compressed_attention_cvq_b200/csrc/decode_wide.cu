@@ -169,7 +169,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   if (warp == 0) stage_codebook(cw_s, kcb, rc, tma_bar);
   stage_codes(t_begin, 0);
   cp_async_commit();
-  for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) bins[i] = 0.f;
+  for (int i = tid; i < kWideCodes * kBinStride / 4; i += kWThreads)
+    reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tid < kWHeads) {
     mref_s[tid] = -INFINITY;
     l_s[tid] = 0.f;
