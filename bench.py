@@ -432,11 +432,11 @@ def run_gpu(args):
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = host_out.numel() * 4 + host_lse.numel() * 4
 
-    # Step i's inputs are copied into one of two device input sets on N_COPY side streams
-    # (each input split into N_COPY byte ranges: one stream moves ~30 GB/s host-to-device on
-    # this box, four ~40) while step i - 1 computes on the other set; the step waits for its
-    # copies, attends, and reads its result back on the main stream.
-    n_copy = 4
+    # Step i's inputs are copied into one of two device input sets on --copy-streams side
+    # streams (inputs of 1 MB and more split into that many byte ranges) while step i - 1
+    # computes on the other set; the step waits for its copies, attends, and reads its
+    # result back on the main stream.
+    n_copy = args.copy_streams
     copy_streams = [torch.cuda.Stream(dev) for _ in range(n_copy)]
     dev_sets = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
     copied = [[torch.cuda.Event() for _ in range(n_copy)] for _ in range(2)]
@@ -601,6 +601,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=workloads.WORKLOAD_ORDER, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--copy-streams", type=int, default=4,
+                    help="host-to-device copy streams of the end-to-end measurement")
     ap.add_argument("--form", choices=["gqa", "gqa_split", "table", "naive"], default="gqa",
                     help="gqa: the library's fast path, one launch; gqa_split: decode and "
                          "combine as two launches; table: the pages' per-query-head table "
