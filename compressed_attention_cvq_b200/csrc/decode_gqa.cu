@@ -440,7 +440,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
                8 * (rank * kLocalGroups + gl2) + d] = v;
     }
   }
-  cluster.sync();   // no CTA leaves while its peer may still address its shared memory
+  // No cluster barrier is needed before leaving: the only distributed-shared-memory access
+  // (the peer's partial-score stores into xchg) precedes the last tile's cluster barrier,
+  // which both CTAs of the pair passed.
   if (a.counters != nullptr) merge_tail(a, b, h, hq0, kHeads, 2 * a.n_splits);
 }
 
