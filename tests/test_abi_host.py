@@ -236,3 +236,9 @@ def test_static_entry_reports_shape_errors():
     st = b.lib.cvq_attend_static(ctypes.byref(_shape(n_q_heads=12)), fake, 0, fake, 0, fake,
                                  fake, fake, fake, 0, 4, fake, fake, None)
     assert st == 2
+
+
+def test_fault_status_rejects_null():
+    # checked before the device is touched
+    assert b.lib.cvq_fault_status(None, 0) == 1
+    assert b.lib.cvq_fault_status(None, 1) == 1
