@@ -242,3 +242,23 @@ def test_fault_status_rejects_null():
     # checked before the device is touched
     assert b.lib.cvq_fault_status(None, 0) == 1
     assert b.lib.cvq_fault_status(None, 1) == 1
+
+
+def test_plain_c_consumer(tmp_path):
+    """cvq.h compiles as strict C99 and a C program links libcvq.so and gets the documented
+    host-side behaviour (tests/c_abi/abi_check.c; nothing it calls launches a kernel)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(b.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    src = os.path.join(ROOT, "tests", "c_abi", "abi_check.c")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), src, "-o", exe, "-L", lib_dir, "-lcvq",
+                    f"-Wl,-rpath,{lib_dir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
