@@ -387,9 +387,11 @@ def run_gpu(args):
     with ClockSampler(local) as clk:
         time.sleep(0.25)   # let the sampler start
         torch.cuda.synchronize()
-        # a fixed-length spin on the GPU (200k cycles, outside the timed region) keeps the stream busy
-        # while the host enqueues the first step, so that step does not include host time
-        torch.cuda._sleep(200_000)
+        # a spin on the GPU (outside the timed region) keeps the stream busy while the host
+        # enqueues the timed steps: ~100 us per step covers the Python and ctypes cost of a
+        # call, so the events measure back-to-back device work even for kernels shorter than
+        # that host cost (the end-to-end leg below includes the host)
+        torch.cuda._sleep(200_000 * (1 + args.steps))
         for i in range(args.steps):
             if i == 0:
                 ev_start.record(stream)

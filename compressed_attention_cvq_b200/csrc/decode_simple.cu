@@ -19,8 +19,20 @@ namespace cvq {
 
 constexpr int kSimpleThreads = 256;
 
-template <int NG, int R, bool TABLE>
+// Threads per token.  TPT = 1: one thread walks a token's 16 groups.  TPT = 4 (for splits of
+// at most kShortSplit tokens): 4 consecutive lanes share a token, lane `part` taking groups
+// 4 part .. 4 part + 3, and a 2-level shuffle adds their partial scores, so a short split
+// keeps all 8 warps busy with a 4x shorter dependent chain per thread.
+constexpr int kShortSplit = 128;
+
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+template <int NG, int R, bool TABLE, int TPT>
 __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const DecodeArgs a) {
+  static_assert(TPT == 1 || TPT == 4, "threads per token");
+  constexpr int kTileTokens = kSimpleThreads / TPT;
   extern __shared__ float4 smem_f4[];
   float* bins = reinterpret_cast<float*>(smem_f4);                // [NG][16][R][256]
   __shared__ float qs[NG][kHeadDim];
@@ -81,8 +93,9 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
   for (int hh = 0; hh < NG; ++hh) { m_run[hh] = -INFINITY; l_run[hh] = 0.f; }
   __syncthreads();
 
-  for (int t0 = t_begin; t0 < t_end; t0 += kSimpleThreads) {
-    const int t = t0 + tid;
+  const int part = tid % TPT;                   // TPT = 4: this lane's groups 4 part .. + 3
+  for (int t0 = t_begin; t0 < t_end; t0 += kTileTokens) {
+    const int t = t0 + tid / TPT;
     const bool valid = t < t_end;
     uint4 kc[R], vc[R];
     float s[NG];
@@ -96,12 +109,16 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
       }
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) s[hh] = 0.f;
+      uint32_t kword[R];                        // TPT = 4: the key code bytes of this lane's groups
+#pragma unroll
+      for (int r = 0; r < R; ++r) kword[r] = word_of(kc[r], part);
 #pragma unroll 4
-      for (int G = 0; G < kGroups; ++G) {
+      for (int gi = 0; gi < kGroups / TPT; ++gi) {
+        const int G = TPT == 1 ? gi : 4 * part + gi;
         float kr[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const int c = code_byte(kc[r], G);
+          const int c = TPT == 1 ? code_byte(kc[r], gi) : static_cast<int>((kword[r] >> (8 * gi)) & 255u);
           const float4* cw = reinterpret_cast<const float4*>(
               tab + ((static_cast<size_t>(G) * R + r) * kCodes + c) * kCodeword);
           const float4 lo = __ldg(cw), hi = __ldg(cw + 1);
@@ -117,6 +134,13 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
 #pragma unroll
           for (int hh = 0; hh < NG; ++hh) s[hh] += qs[hh][2 * j] * xr + qs[hh][2 * j + 1] * xi;
         }
+      }
+    }
+    if constexpr (TPT > 1) {                    // add the partial scores of the token's lanes
+#pragma unroll
+      for (int o = 1; o < TPT; o <<= 1) {
+#pragma unroll
+        for (int hh = 0; hh < NG; ++hh) s[hh] += __shfl_xor_sync(0xffffffffu, s[hh], o);
       }
     }
     // tile max per head
@@ -153,13 +177,16 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) {
         const float w = exp2f(s[hh] - m_run[hh]);
-        l_run[hh] += w;
+        if (part == 0) l_run[hh] += w;          // once per token
         float* bh = bins + hh * kGroups * R * kCodes;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
+          const uint32_t vword = word_of(vc[r], part);
 #pragma unroll
-          for (int G = 0; G < kGroups; ++G) {
-            atomicAdd(bh + (G * R + r) * kCodes + code_byte(vc[r], G), w);
+          for (int gi = 0; gi < kGroups / TPT; ++gi) {
+            const int G = TPT == 1 ? gi : 4 * part + gi;
+            const int c = TPT == 1 ? code_byte(vc[r], gi) : static_cast<int>((vword >> (8 * gi)) & 255u);
+            atomicAdd(bh + (G * R + r) * kCodes + c, w);
           }
         }
       }
@@ -249,7 +276,8 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
 template <int NG, int R, bool TABLE>
 static cudaError_t launch_simple(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(NG) * kGroups * R * kCodes * sizeof(float);
-  auto k = decode_simple_kernel<NG, R, TABLE>;
+  auto k = a.split_tokens <= kShortSplit ? decode_simple_kernel<NG, R, TABLE, 4>
+                                         : decode_simple_kernel<NG, R, TABLE, 1>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
