@@ -184,8 +184,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned i
 // the arithmetic of combine_kernel, in the same order, and clears the counter for the
 // next call.  No CTA waits for another: the others simply finish.  The arrival is one
 // acq_rel atomic per CTA (measured 0.5-1 us faster than a full fence before a relaxed one).
+// W warps per query head (n_heads * W <= blockDim / 32): lane l of the head's warp w owns
+// the 4 / W output dims 32 w + l + 32 W j and sums them over the splits in split order, as
+// combine_kernel does per dim, so both give the same bits; loads go U splits at a time, one
+// group ahead of their use.
+template <int W = 1, int U = 4>
 __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit, int hq0,
                                            int n_heads, int expected) {
+  static_assert(W == 1 || W == 2 || W == 4, "warps per head");
+  constexpr int D = 4 / W;                         // output dims per lane
   int* ctr = a.counters + static_cast<size_t>(b) * gridDim.y + unit;
   int old = 0;
   __syncthreads();                       // this CTA's partial states are all written
@@ -195,24 +202,22 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
   }
   if (!__syncthreads_or(threadIdx.x == 0 && old == expected - 1)) return;
-  // One warp per query head; lane l owns output dims l, l + 32, l + 64, l + 96.  Loads are
-  // issued 4 splits at a time, one group ahead of its use (they do not depend on M), and the
-  // sums run over the splits in order, as in combine_kernel.
-  constexpr int kU = 4;
+  constexpr int kU = U;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.n_splits;
-  for (int hh = warp; hh < n_heads; hh += blockDim.x >> 5) {
+  const int wl = warp % W;
+  for (int hh = warp / W; hh < n_heads; hh += (blockDim.x >> 5) / W) {
     const size_t row = static_cast<size_t>(b) * a.n_q_heads + hq0 + hh;
     const float* pm = a.part_m + row * S;
     const float* pl = a.part_l + row * S;
-    const float* po = a.part_o + row * S * kHeadDim + lane;
-    float x[kU][4];
+    const float* po = a.part_o + row * S * kHeadDim + 32 * wl + lane;
+    float x[kU][D];
     auto load_o = [&](int s0) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          x[u][j] = s0 + u < S ? __ldcg(po + static_cast<size_t>(s0 + u) * kHeadDim + 32 * j) : 0.f;
+        for (int j = 0; j < D; ++j)
+          x[u][j] = s0 + u < S ? __ldcg(po + static_cast<size_t>(s0 + u) * kHeadDim + 32 * W * j) : 0.f;
       }
     };
     float mv = lane < S ? __ldcg(pm + lane) : -INFINITY;    // splits 0..31
@@ -222,25 +227,27 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
     for (int s = lane + 32; s < S; s += 32) M = fmaxf(M, __ldcg(pm + s));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float* orow = a.out + row * kHeadDim + lane;
+    float* orow = a.out + row * kHeadDim + 32 * wl + lane;
     if (M == -INFINITY) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) orow[32 * j] = 0.f;
-      if (lane == 0) a.lse[row] = -INFINITY;
+      for (int j = 0; j < D; ++j) orow[32 * W * j] = 0.f;
+      if (wl == 0 && lane == 0) a.lse[row] = -INFINITY;
       continue;
     }
-    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = 0.f, acc[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) acc[j] = 0.f;
     for (int s0 = 0; s0 < S; s0 += kU) {                      // splits in order
       if (s0 % 32 == 0 && s0 > 0) {                          // next 32 splits' m and l
         mv = s0 + lane < S ? __ldcg(pm + s0 + lane) : -INFINITY;
         lv = s0 + lane < S ? __ldcg(pl + s0 + lane) : 0.f;
       }
       const float fv = (mv == -INFINITY) ? 0.f : expf(mv - M);
-      float y[kU][4];
+      float y[kU][D];
 #pragma unroll
       for (int u = 0; u < kU; ++u)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) y[u][j] = x[u][j];
+        for (int j = 0; j < D; ++j) y[u][j] = x[u][j];
       if (s0 + kU < S) load_o(s0 + kU);                       // the next group, in flight
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
@@ -249,13 +256,13 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
           const float f = __shfl_sync(0xffffffffu, fv, src);
           L = fmaf(__shfl_sync(0xffffffffu, lv, src), f, L);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[j] = fmaf(y[u][j], f, acc[j]);
+          for (int j = 0; j < D; ++j) acc[j] = fmaf(y[u][j], f, acc[j]);
         }
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) orow[32 * j] = acc[j] / L;
-    if (lane == 0) a.lse[row] = M + logf(L);
+    for (int j = 0; j < D; ++j) orow[32 * W * j] = acc[j] / L;
+    if (wl == 0 && lane == 0) a.lse[row] = M + logf(L);
   }
   if (threadIdx.x == 0) atomicExch(ctr, 0);
 }

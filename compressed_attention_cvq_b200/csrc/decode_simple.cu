@@ -32,6 +32,8 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
 template <int NG, int R, bool TABLE, int TPT>
 __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const DecodeArgs a) {
   static_assert(TPT == 1 || TPT == 4, "threads per token");
+  // warps per query head in the fused merge
+  constexpr int kMergeW = (kSimpleThreads / 32) / NG >= 4 ? 4 : (kSimpleThreads / 32) / NG;
   constexpr int kTileTokens = kSimpleThreads / TPT;
   extern __shared__ float4 smem_f4[];
   float* bins = reinterpret_cast<float*>(smem_f4);                // [NG][16][R][256]
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
       a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
     }
     if constexpr (!TABLE) {   // the fused merge serves cvq_attend (GQA form) only
-      if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+      if (a.counters != nullptr) merge_tail<kMergeW, 4 * kMergeW>(a, b, head, hq0, NG, a.n_splits);
     }
     return;
   }
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
     }
   }
   if constexpr (!TABLE) {
-    if (a.counters != nullptr) merge_tail(a, b, head, hq0, NG, a.n_splits);
+    if (a.counters != nullptr) merge_tail<kMergeW, 4 * kMergeW>(a, b, head, hq0, NG, a.n_splits);
   }
 }
 
