@@ -1,6 +1,7 @@
 // Split-T flash-decode over the uint8 code stream: the straightforward form.
 //
-// One CTA = (split, head, sequence); one thread = one token of a 256-token tile.
+// One CTA = (split, head, sequence); one thread = one token of a 256-token tile (on splits
+// of at most 128 tokens: 4 threads = one token of a 64-token tile, see TPT below).
 // Per token: gather the key codewords of every (group, round) from the table
 // (global memory, L1/L2 cached), sum the rounds, rotate by the RoPE phase
 // e^{i theta_j t} and project on the query head(s) -> score (in log2 units).
