@@ -32,12 +32,13 @@ __all__ = ["make_shape", "shape_of", "qtable", "decode_attn", "decode_attn_gqa",
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    # a plain int (or None) converts to the c_void_p argument without a ctypes object
+    return t.data_ptr() if t is not None else None
 
 
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    return s.cuda_stream
 
 
 def _require(t, name, dtype=None, device=True):

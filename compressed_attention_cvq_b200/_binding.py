@@ -75,7 +75,9 @@ class _LazyLib:
     def __getattr__(self, name):
         if _LazyLib._lib is None:
             _LazyLib._lib = _load()
-        return getattr(_LazyLib._lib, name)
+        fn = getattr(_LazyLib._lib, name)
+        setattr(self, name, fn)          # later lookups skip __getattr__
+        return fn
 
 
 lib = _LazyLib()

@@ -4,6 +4,7 @@
 
 #include <cuda.h>            // CUtensorMap (the type only; the encoder is reached at run time)
 #include <cuda_runtime.h>
+#include <atomic>
 #include <stdint.h>
 
 #include "cvq.h"
@@ -286,6 +287,33 @@ cudaError_t launch_naive_decode(const cvq_shape& s, const void* q, int q_dtype, 
                                 cudaStream_t stream);
 // 64-scalar groups, 4 query heads per KV head (decode_wide.cu)
 cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream);
+
+// The dynamic-shared-memory limit of a kernel is a per-device setting: apply it once per
+// (kernel, device) instead of on every launch.  `flag` is a static of the calling launcher,
+// one per kernel; devices 0..127.
+class PerDeviceFlag {
+ public:
+  bool done(int dev) const {
+    return dev >= 0 && dev < 128 && ((bits_[dev >> 6].load(std::memory_order_acquire) >> (dev & 63)) & 1u);
+  }
+  void mark(int dev) {
+    if (dev >= 0 && dev < 128) bits_[dev >> 6].fetch_or(1ull << (dev & 63), std::memory_order_release);
+  }
+
+ private:
+  std::atomic<unsigned long long> bits_[2] = {};
+};
+
+template <typename Kernel>
+cudaError_t set_smem_limit_once(PerDeviceFlag& flag, Kernel kernel, size_t bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (flag.done(dev)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) flag.mark(dev);
+  return e;
+}
 
 // Host side of the TMA staging and the fault word (device_state.cu).
 // Tiled map of one codebook tensor (key or value, narrow layout: per head [16 groups][R][256

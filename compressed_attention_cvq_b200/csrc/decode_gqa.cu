@@ -450,8 +450,8 @@ template <int R>
 cudaError_t launch_gqa4(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = Cfg<R>::kSmem;
   auto k = decode_gqa4_kernel<R>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static PerDeviceFlag smem_set;
+  cudaError_t e = set_smem_limit_once(smem_set, k, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.n_splits, s.n_kv_heads, s.batch);
   k<<<grid, Cfg<R>::kThreads, smem, stream>>>(a);

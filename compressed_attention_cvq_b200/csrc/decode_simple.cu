@@ -279,10 +279,10 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
 template <int NG, int R, bool TABLE>
 static cudaError_t launch_simple(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(NG) * kGroups * R * kCodes * sizeof(float);
-  auto k = a.split_tokens <= kShortSplit ? decode_simple_kernel<NG, R, TABLE, 4>
-                                         : decode_simple_kernel<NG, R, TABLE, 1>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const bool short_split = a.split_tokens <= kShortSplit;
+  auto k = short_split ? decode_simple_kernel<NG, R, TABLE, 4> : decode_simple_kernel<NG, R, TABLE, 1>;
+  static PerDeviceFlag smem_set_short, smem_set_long;
+  cudaError_t e = set_smem_limit_once(short_split ? smem_set_short : smem_set_long, k, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, TABLE ? s.n_q_heads : s.n_kv_heads, s.batch);
   k<<<grid, kSimpleThreads, smem, stream>>>(a);

@@ -392,9 +392,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 
 cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
   const int C = wide_cluster_size(s.R);
-  cudaError_t e = cudaFuncSetAttribute(decode_wide_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kWSmem));
+  static PerDeviceFlag smem_set;
+  cudaError_t e = set_smem_limit_once(smem_set, decode_wide_kernel, kWSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.n_splits * C), s.n_kv_heads, s.batch);

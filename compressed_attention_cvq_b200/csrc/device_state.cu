@@ -50,8 +50,32 @@ cudaError_t encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
 
 namespace cvq {
 
+// A map depends only on (base, head stride, heads, R): the last kMapCache maps encoded are
+// kept, so a decode loop over the same codebooks does not re-encode them every call.
+namespace {
+constexpr int kMapCache = 16;
+struct MapEntry {
+  const float* base = nullptr;
+  long long head_stride = 0;
+  int n_heads = 0, R = 0;
+  bool valid = false;
+  CUtensorMap map;
+};
+MapEntry g_map_cache[kMapCache];
+int g_map_next = 0;
+}  // namespace
+
 cudaError_t encode_codebook_map(CUtensorMap* map, const float* base, long long head_stride,
                                 int n_heads, int R) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (const MapEntry& m : g_map_cache) {
+      if (m.valid && m.base == base && m.head_stride == head_stride && m.n_heads == n_heads && m.R == R) {
+        *map = m.map;
+        return cudaSuccess;
+      }
+    }
+  }
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -68,7 +92,17 @@ cudaError_t encode_codebook_map(CUtensorMap* map, const float* base, long long h
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides,
                          box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lock(g_mu);
+  MapEntry& slot = g_map_cache[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCache;
+  slot.base = base;
+  slot.head_stride = head_stride;
+  slot.n_heads = n_heads;
+  slot.R = R;
+  slot.map = *map;
+  slot.valid = true;
+  return cudaSuccess;
 }
 
 cudaError_t fault_word_address(unsigned int** out) {

@@ -125,8 +125,8 @@ cudaError_t launch_nv(const cvq_shape& s, const void* q, int q_dtype, const void
                       float* pm, float* pl, cudaStream_t stream) {
   const size_t smem = sizeof(float) * kStreams * NG * (kHeadDim + 2);
   auto kern = naive_decode_kernel<NG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static PerDeviceFlag smem_set;
+  cudaError_t e = set_smem_limit_once(smem_set, kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(n_splits, s.n_kv_heads, s.batch);
   kern<<<grid, kNvThreads, smem, stream>>>(q, q_dtype, static_cast<const __half*>(k),

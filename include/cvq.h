@@ -42,6 +42,10 @@
  *   - The first GQA decode call on a device (cvq_decode_attn_gqa, cvq_attend,
  *     cvq_attend_static) looks up the device fault word's address with that device
  *     current; make it before any stream capture.
+ *   - Per device, the library remembers the device addresses of its own device variables
+ *     (fault word, static scratch) and the shared-memory limit it set on each kernel.  Like
+ *     any state tied to a CUDA context, these do not survive cudaDeviceReset: do not call
+ *     the library on a device after resetting it in the same process.
  */
 #ifndef CVQ_H
 #define CVQ_H
