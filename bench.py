@@ -68,11 +68,14 @@ def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
 
 def encode_work(w: workloads.Workload):
     """Algorithmic work of one append (every sequence and KV head, key and value): per
-    group and round, 256 codewords x 8 dims x (sub, mul, add) FLOP; bytes = both codebooks
+    group and round, every codeword x the group's dims x (sub, mul, add) FLOP (16 groups x
+    256 codewords x 8 dims, or 2 x 64 x 64 with 64-scalar groups); bytes = both codebooks
     of every KV head + the new vectors + the written codes."""
     units = w.batch * w.n_kv_heads
-    flops = float(units) * 2 * 16 * w.R * 256 * 8 * 3
-    bytes_ = 2.0 * w.n_kv_heads * 16 * w.R * 256 * 8 * 4 + units * (2 * 128 * 4 + 2 * 16 * w.R)
+    per_round = w.n_groups * w.n_codes * w.group_dim
+    flops = float(units) * 2 * w.R * per_round * 3
+    bytes_ = (2.0 * w.n_kv_heads * w.R * per_round * 4
+              + units * (2 * 128 * 4 + 2 * w.n_groups * w.R))
     return flops, bytes_
 
 

@@ -1,0 +1,61 @@
+"""Host-side checks of bench.py's accounting (no GPU): the algorithmic FLOPs and bytes per
+layer step, the shared-memory floor, the append work and the whole-job rate, each against a
+value worked out by hand from the definitions in the docstrings (per token and query head:
+64 pairs x (2 mul + 2 add) = 256 FLOP, + 128 (R - 1) to sum rounds, + one bin add per
+(group, round); per token and KV head: one code byte per (group, round) for keys and for
+values)."""
+import math
+
+import pytest
+
+import bench
+import workloads
+
+W = workloads.WORKLOADS
+
+
+def test_algorithmic_flops_by_hand():
+    # 128K layer, R = 1: 131072 tokens x 32 heads x (256 + 0 + 16)
+    assert bench.algorithmic_flops(W["llama8b_layer_T131072_R1"], 131072) == 131072 * 32 * 272
+    # 32K layer, R = 2: 256 + 128 + 32 = 416 per token and head
+    assert bench.algorithmic_flops(W["llama8b_layer_T32768_R2"], 32768) == 32768 * 32 * 416
+    # paper's 1-bit setting, R = 11 over 2 groups: 256 + 1280 + 22 = 1558
+    assert bench.algorithmic_flops(W["llama8b_layer_T131072_R11_g64"], 131072) == 131072 * 32 * 1558
+
+
+def test_code_bytes_by_hand():
+    # 128K layer, R = 1: codes 131072 x 8 KV heads x (16 key + 16 value bytes) = 33,554,432;
+    # codebooks 2 x 8 heads x 16 groups x 256 codewords x 8 floats x 4 B = 2,097,152
+    assert bench.code_bytes(W["llama8b_layer_T131072_R1"], 131072) == 33_554_432 + 2_097_152
+    # R = 11 over 64-scalar groups: codes 131072 x 8 x 2 x 2 x 11; codebooks
+    # 2 x 8 x 2 groups x 11 rounds x 64 codewords x 64 floats x 4 B
+    assert bench.code_bytes(W["llama8b_layer_T131072_R11_g64"], 131072) == (
+        131072 * 8 * 2 * 2 * 11 + 2 * 8 * 2 * 11 * 64 * 64 * 4)
+
+
+def test_smem_floor_by_hand():
+    # per token and KV head at R = 1: 512 B of codewords at 125.6 B/clk and 16 groups x 4
+    # heads of bin atomics at 7.73 lanes/clk, over 148 SMs at 1965 MHz
+    clk = 512 / 125.6 + 64 / 7.73
+    expect = 131072 * 8 * clk / 148 / 1965
+    got = bench.smem_floor_us(W["llama8b_layer_T131072_R1"], 131072, 1965.0)
+    assert math.isclose(got, expect, rel_tol=1e-12)
+    assert 44.0 < got < 45.0
+
+
+def test_encode_work_by_hand():
+    # one append on the 128K layer (B = 1, 8 KV heads, R = 1): key and value, 16 groups x
+    # 256 codewords x 8 dims x 3 FLOP each; bytes = both codebooks + the new vectors + codes
+    flops, bytes_ = bench.encode_work(W["llama8b_layer_T131072_R1"])
+    assert flops == 8 * 2 * 16 * 256 * 8 * 3
+    assert bytes_ == 2 * 8 * 16 * 256 * 8 * 4 + 8 * (2 * 128 * 4 + 2 * 16)
+    # 64-scalar groups, R = 11: 2 groups x 64 codewords x 64 dims per round
+    flops, bytes_ = bench.encode_work(W["llama8b_layer_T131072_R11_g64"])
+    assert flops == 8 * 2 * 11 * 2 * 64 * 64 * 3
+    assert bytes_ == 2 * 8 * 11 * 2 * 64 * 64 * 4 + 8 * (2 * 128 * 4 + 2 * 2 * 11)
+
+
+@pytest.mark.parametrize("world,units,ms,expect", [(1, 131072, 0.15, 131072 / 0.15e-3),
+                                                   (4, 1000, 2.0, 4 * 1000 / 2e-3)])
+def test_whole_job_rate(world, units, ms, expect):
+    assert math.isclose(bench.whole_job_rate(world, units, ms), expect, rel_tol=1e-12)
