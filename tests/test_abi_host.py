@@ -262,3 +262,26 @@ def test_plain_c_consumer(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert "c abi ok" in r.stdout
+
+
+def test_attend_more_argument_errors():
+    """Further cvq_attend argument errors, each caught on the host before the device is
+    touched: split count range, alignments, query dtype, RoPE base, group size, batch."""
+    def call(shape, n_splits=4, q_dtype=0, **kw):
+        a = dict(q=FAKE, kcb=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, vcb=FAKE, ws=FAKE, out=FAKE,
+                 lse=FAKE)
+        a.update(kw)
+        return b.lib.cvq_attend(ctypes.byref(shape), a["q"], q_dtype, a["kcb"], 0, a["kc"],
+                                a["vc"], a["lens"], a["vcb"], 0, n_splits, a["ws"], a["out"],
+                                a["lse"], None)
+    s = _shape()
+    assert call(s, n_splits=0) == 5
+    assert call(s, n_splits=4097) == 5
+    assert call(s, lse=FAKE + 2) == 3
+    assert call(s, lens=FAKE + 2) == 3
+    assert call(s, q_dtype=7) == 4
+    assert call(_shape(rope_base=1.0)) == 2
+    assert call(_shape(rope_base=float("nan"))) == 2
+    assert call(_shape(n_q_heads=24, n_kv_heads=8)) == 4          # 3 query heads per KV head
+    assert call(_shape(n_q_heads=30, n_kv_heads=8)) == 2          # not a multiple
+    assert call(_shape(batch=70000)) == 2
