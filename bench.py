@@ -43,9 +43,14 @@ import workloads  # noqa: E402
 
 DEFAULT_WORKLOAD = "llama8b_layer_T131072_R1"
 METRIC = "CommVQ decode attn: KV tokens/s per layer; code HBM GB/s vs B200 peak"
-FP32_LANES_PER_SM = 128
 SM_COUNT_B200 = 148
 N_INPUT_SETS = 8
+# Unit throughputs measured on B200 by compressed_attention_cvq_b200.microbench (per SM per
+# clock, 1965 MHz): FP32 FMA lanes, sin+cos pairs (__sincosf) and exp2 results.
+FFMA_LANES_PER_CLK = 123.74
+SINCOS_PAIRS_PER_CLK = 7.95
+EXP2_PER_CLK = 15.90
+SUSTAINED_S = 1.5            # device time of the sustained loop after the timed steps
 
 
 def algorithmic_flops(w: workloads.Workload, total_tokens: int) -> float:
@@ -55,6 +60,25 @@ def algorithmic_flops(w: workloads.Workload, total_tokens: int) -> float:
     the SFU, not here)."""
     per_tok_head = 256 + 128 * (w.R - 1) + w.n_groups * w.R
     return float(total_tokens) * w.n_q_heads * per_tok_head
+
+
+def sfu_ops(w: workloads.Workload, total_tokens: int):
+    """Algorithmic special-function work of one layer step: the RoPE phase of every pair
+    once per token and sequence (64 sin+cos pairs, shared by all heads) and one exp per
+    token and query head."""
+    return float(total_tokens) * 64, float(total_tokens) * w.n_q_heads
+
+
+def roofline_legs(w: workloads.Workload, total_tokens: int, sm_mhz: float, hbm_gbs: float):
+    """Time (us) of one layer step at each bound: FP32 work at the measured FFMA rate, the
+    special-function work at the measured sin/cos and exp2 rates, and the code + codebook
+    bytes at the measured HBM copy bandwidth.  The roofline is the slowest of the three."""
+    clk_hz = SM_COUNT_B200 * sm_mhz * 1e6
+    fp32_us = algorithmic_flops(w, total_tokens) / 2 / FFMA_LANES_PER_CLK / clk_hz * 1e6
+    sc, ex = sfu_ops(w, total_tokens)
+    sfu_us = (sc / SINCOS_PAIRS_PER_CLK + ex / EXP2_PER_CLK) / clk_hz * 1e6
+    hbm_us = code_bytes(w, total_tokens) / (hbm_gbs * 1e9) * 1e6
+    return {"fp32_us": fp32_us, "sfu_us": sfu_us, "hbm_us": hbm_us}
 
 
 def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
@@ -116,8 +140,8 @@ def append_summary(w: workloads.Workload, enc_ms):
 
 def recorded_traffic(workload: str, form: str):
     """DRAM bytes per launch of the decode kernel from the committed ncu record, if it was
-    taken on this workload and form and none of the kernel's sources has changed since
-    (else None)."""
+    taken on this workload and form and none of the kernel's device sources (the kernel's
+    own file and the shared device header) has changed since (else None)."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -153,6 +177,13 @@ def parity_of(layer0, outputs):
         el = max(el, abs(float(lse[b, hq]) - rl) / max(abs(rl), 1.0))
     return {"heads": len(outputs), "max_abs_err": eo, "lse_rel_err": el,
             "tolerance": {"max_abs_err": 2e-3, "lse_rel_err": 1e-4}}
+
+
+def workload_config(w: workloads.Workload, args, total_tokens: int) -> dict:
+    """The workload a line measures, identical in the GPU arm and the reference arm."""
+    return {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R, "group_dim": w.group_dim,
+            "q_dtype": w.q_dtype, "tokens_per_layer": total_tokens, "append": bool(args.append)}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -277,7 +308,7 @@ def oracle_sample(w: workloads.Workload, budget_s: float = 12.0, layer: int = 0)
     # one layer = every query head over its sequence: scale the token-heads done
     layer_time = el * (total_tokens * w.n_q_heads) / max(done_tokens, 1)
     return {"value": total_tokens / layer_time, "unit": "KV tokens/s per layer", "cores": 1,
-            "kind": "oracle",
+            "kind": "oracle", "heads": n, "elapsed_s": el,
             "sample": f"{n} of {len(heads)} (sequence, query head) pairs of layer {layer} "
                       f"({done_tokens} token-heads, {el:.1f} s), scaled to the full layer",
             "seconds_per_layer": layer_time, "outputs": outputs}
@@ -286,6 +317,51 @@ def oracle_sample(w: workloads.Workload, budget_s: float = 12.0, layer: int = 0)
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def sustained_run(step, args, n_sets, stream, dev):
+    """Replay a CUDA graph of n_sets consecutive steps until about SUSTAINED_S seconds of
+    device time have passed; per-step device time from one event pair per replay."""
+    import torch
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(n_sets):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    est_ms = max(t0.elapsed_time(t1) / n_sets, 1e-3)
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(n_sets):
+                    step(i)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        via = f"CUDA graph of {n_sets} steps, replayed"
+        run = g.replay
+    except Exception as e:  # noqa: BLE001 - report and enqueue directly instead
+        g = None
+        via = f"direct enqueue ({type(e).__name__} while capturing)"
+
+        def run():
+            for i in range(n_sets):
+                step(i)
+    reps = max(1, int(math.ceil(SUSTAINED_S * 1e3 / (est_ms * n_sets))))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    torch.cuda.synchronize()
+    evs[0].record(stream)
+    for r in range(reps):
+        run()
+        evs[r + 1].record(stream)
+    torch.cuda.synchronize()
+    per_rep = [evs[r].elapsed_time(evs[r + 1]) / n_sets for r in range(reps)]
+    del g
+    return {"steps": reps * n_sets, "device_s": sum(per_rep) * n_sets / 1e3,
+            "ms_per_step_mean": statistics.mean(per_rep),
+            "ms_per_step_median": statistics.median(per_rep), "via": via}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -400,6 +476,11 @@ def run_gpu(args):
                 ev_start.record(stream)
             step(args.warmup + i, evs[i])
         torch.cuda.synchronize()
+        # Sustained load: the same step for ~SUSTAINED_S s of device time right after the
+        # timed steps, so that the clock sampler sees the kernel under load for many samples.
+        # The steps (one per input set) are captured once in a CUDA graph and replayed, so
+        # the host's enqueue cost does not gate short kernels.
+        sustained = sustained_run(step, args, n_sets, stream, dev)
     if world > 1:
         dist.barrier()
     starts = [ev_start] + [e["end"] for e in evs[:-1]]
@@ -515,7 +596,10 @@ def run_gpu(args):
         pk, pk_src = peaks()
         dec_mean_ms = statistics.mean(dec_ms)
         sm_max = pk.get("sm_max_mhz", 1965.0) or 1965.0
-        fp32_peak_tflops = SM_COUNT_B200 * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+        fp32_peak_tflops = SM_COUNT_B200 * FFMA_LANES_PER_CLK * 2 * sm_max * 1e6 / 1e12
+        legs = roofline_legs(w, total_tokens, sm_max, pk["hbm_gbs"])
+        bound_leg = max(legs, key=legs.get)
+        bound = {"fp32_us": "alu", "sfu_us": "sfu", "hbm_us": "hbm"}[bound_leg]
         flops = algorithmic_flops(w, total_tokens)
         achieved_tflops = flops / (dec_mean_ms * 1e-3) / 1e12
         bytes_ = code_bytes(w, total_tokens)
@@ -533,29 +617,32 @@ def run_gpu(args):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic (seeded codebooks, codes and queries; no trained weights)",
-            "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
-                       "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R,
-                       "q_dtype": w.q_dtype, "form": args.form, "n_splits": S,
-                       "append": bool(args.append),
-                       "tokens_per_layer": total_tokens,
-                       "l2": f"{N_INPUT_SETS} rotating layer input sets of "
-                             f"{code_bytes(w, total_tokens) / 1e6:.0f} MB (> 126 MB L2 in total)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": workload_config(w, args, total_tokens),
+            "run": {"form": args.form, "n_splits": S,
+                    "l2": f"{N_INPUT_SETS} rotating layer input sets of "
+                          f"{code_bytes(w, total_tokens) / 1e6:.0f} MB (> 126 MB L2 in total)",
+                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "decode_ms": dec_mean_ms,
             "decode_ms_median": statistics.median(dec_ms),
             "step_ms_median": statistics.median(step_ms),
             "code_hbm_gbs": bytes_ / (dec_mean_ms * 1e-3) / 1e9,
             "code_hbm_frac": bytes_ / (dec_mean_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-            "roofline": {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak_tflops,
-                         "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
+            "roofline": {"bound": bound, "achieved": achieved_tflops, "peak": fp32_peak_tflops,
+                         "unit": "TFLOP/s", "frac": legs[bound_leg] / (dec_mean_ms * 1e3),
                          "traffic": recorded_traffic(args.workload, args.form),
                          "traffic_unit": "DRAM bytes per decode launch (ncu)",
-                         "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {sm_max:.0f} MHz "
-                                        f"(unit counts and max clock; HBM peak {pk_src})"},
+                         "legs_us": legs,
+                         "peak_source": f"148 SMs x {FFMA_LANES_PER_CLK} FFMA lanes/clk x 2 x "
+                                        f"{sm_max:.0f} MHz (measured FFMA rate, "
+                                        f"compressed_attention_cvq_b200.microbench); SFU leg at "
+                                        f"{SINCOS_PAIRS_PER_CLK} sin+cos pairs and {EXP2_PER_CLK} "
+                                        f"exp2 per SM-clock (measured); HBM {pk['hbm_gbs']} GB/s "
+                                        f"({pk_src})"},
             "e2e": {"value": whole_job_rate(world, total_tokens, e2e_ms), "unit": "KV tokens/s per layer",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "smem_floor": smem_summary(w, total_tokens, dec_mean_ms, pk, args.form),
             "gpu_launches": args.steps * launches_per_step,
+            "sustained": sustained,
             "device_faults": fault,
             "_layer0": layer0,
             "append": append_summary(w, enc_ms) if args.append else None,
@@ -575,27 +662,35 @@ def run_reference(args):
     per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(w, budget_s=min(per_step, 5.0))
-    vals = []
+    vals, last_s = [], []
     t0 = time.perf_counter()
     last = None
     for i in range(args.steps):
         last = oracle_sample(w, budget_s=per_step, layer=0)
         vals.append(last["value"])
+        last_s.append(last["elapsed_s"])
     el = time.perf_counter() - t0
     value = statistics.mean(vals)
     total_tokens = int(workloads.make_seq_lens(w).sum())
     return {
         "metric": METRIC, "impl": "reference", "value": value, "unit": "KV tokens/s per layer",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * total_tokens / value, "higher_is_better": True, "scaling": "weak",
+        # one step = one full layer pass; each step timed only a sample of its (sequence,
+        # query head) pairs and was scaled linearly to the layer (extrapolated)
+        "ms_per_step": 1e3 * total_tokens / value,
+        "ms_per_step_extrapolated": True,
+        "extrapolated_from_s": sum(last_s) / len(last_s),
+        "sampled_heads_per_step": last["heads"],
+        "heads_per_layer": w.batch * w.n_q_heads,
+        "measured_wall_s": el,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
-                   "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R, "q_dtype": w.q_dtype},
+        "config": workload_config(w, args, total_tokens),
+        "run": {"form": "oracle", "parallelism": "1 host core"},
         "cpu_baseline": {"value": value, "unit": "KV tokens/s per layer", "cores": 1, "kind": "oracle",
                          "sample": f"each step: {last['sample']}"},
         "e2e": {"value": value, "unit": "KV tokens/s per layer", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
-        "wall_s": el,
     }
 
 

@@ -111,7 +111,8 @@ cvq_status decode_gqa_impl(const cvq_shape* s, const void* q, int q_dtype, const
                            int64_t key_cb_head_stride, const uint8_t* key_codes,
                            const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
                            int64_t val_cb_head_stride, int n_splits, float* part_o, float* part_m,
-                           float* part_l, int* counters, float* out, float* lse, void* stream) {
+                           float* part_l, int* counters, float* out, float* lse, void* stream,
+                           size_t clear_counters = 0) {
   CVQ_TRY(check_shape(s));
   if (q_dtype != CVQ_F32 && q_dtype != CVQ_BF16) return CVQ_ERR_UNSUPPORTED;
   CVQ_TRY(check_ptr(q));
@@ -139,6 +140,12 @@ cvq_status decode_gqa_impl(const cvq_shape* s, const void* q, int q_dtype, const
         encode_codebook_map(&a.val_map, val_cb, val_cb_head_stride, s->n_kv_heads, s->R) != cudaSuccess)
       return CVQ_ERR_CUDA;
   }
+  // every argument is valid: clear the counters first if the caller asked (enqueued on the
+  // same stream, so the decode kernel sees them zero)
+  if (clear_counters != 0 &&
+      cudaMemsetAsync(counters, 0, clear_counters * sizeof(int), static_cast<cudaStream_t>(stream)) !=
+          cudaSuccess)
+    return CVQ_ERR_CUDA;
   if (is_wide(s)) return from_cuda(launch_decode_wide(*s, a, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_decode_gqa(*s, a, static_cast<cudaStream_t>(stream)));
 }
@@ -163,6 +170,29 @@ void phase_turns_host(float rope_base, PhaseTurns* out) {
     }
     out->F[j] = f;
   }
+}
+
+cvq_status attend_into(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                       int64_t key_cb_head_stride, const uint8_t* key_codes,
+                       const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                       int64_t val_cb_head_stride, int n_splits, float* partials, int* counters,
+                       float* out, float* lse, void* stream, size_t clear_counters) {
+  CVQ_TRY(check_shape(s));
+  CVQ_TRY(check_ptr(partials));
+  if (counters == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(counters) & 3u) != 0) return CVQ_ERR_ALIGN;
+  CVQ_TRY(check_ptr(out));
+  if (lse == nullptr) return CVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return CVQ_ERR_ALIGN;
+  if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
+  // partials: part_o [rows][128], part_m [rows], part_l [rows]
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
+  float* part_o = partials;
+  float* part_m = part_o + rows * kHeadDim;
+  float* part_l = part_m + rows;
+  return decode_gqa_impl(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
+                         seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
+                         counters, out, lse, stream, clear_counters);
 }
 
 }  // namespace cvq
@@ -290,14 +320,11 @@ cvq_status cvq_attend(const cvq_shape* s, const void* q, int q_dtype, const floa
   if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
   // workspace: part_o [rows][128], part_m [rows], part_l [rows], then the counters
   const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * n_splits;
-  float* part_o = static_cast<float*>(workspace);
-  float* part_m = part_o + rows * kHeadDim;
-  float* part_l = part_m + rows;
   int* counters = reinterpret_cast<int*>(static_cast<char*>(workspace) +
                                          round16(rows * (kHeadDim + 2) * sizeof(float)));
-  return decode_gqa_impl(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
-                         seq_lens, val_cb, val_cb_head_stride, n_splits, part_o, part_m, part_l,
-                         counters, out, lse, stream);
+  return cvq::attend_into(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes,
+                          seq_lens, val_cb, val_cb_head_stride, n_splits,
+                          static_cast<float*>(workspace), counters, out, lse, stream, 0);
 }
 
 cvq_status cvq_combine(const cvq_shape* s, int n_splits, const float* part_o, const float* part_m,

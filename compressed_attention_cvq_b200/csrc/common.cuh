@@ -119,10 +119,9 @@ constexpr unsigned int kFaultCopyTimeout = CVQ_FAULT_COPY_TIMEOUT;   // a TMA co
 constexpr int kCodeBoxRows = 32;   // codes per TMA box of the codebook maps
 
 // ---- mbarrier + TMA (bulk copy engine) helpers ----
-// try_wait rounds before a wait gives up; each round suspends the thread for at most about
-// the hint below (ns), so the limit is a few seconds
-constexpr int kMbarTries = 1 << 22;
-constexpr unsigned int kMbarSuspendNs = 1000u;
+// A bounded wait polls the barrier (try_wait, no suspend hint) and gives up once this many
+// nanoseconds of %globaltimer have passed since its first poll.
+constexpr unsigned long long kMbarWaitLimitNs = 2000000000ull;   // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -152,7 +151,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned int parity) {
     unsigned long long now;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
     if (i == 0) t0 = now;
-    else if (now - t0 > 2000000000ull) return false;
+    else if (now - t0 > kMbarWaitLimitNs) return false;
   }
 }
 // order this thread's earlier generic-proxy shared-memory accesses before later TMA writes
@@ -328,6 +327,16 @@ cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const fl
                                  const float* key_cb, long long key_stride, const float* val_cb,
                                  long long val_stride, const int32_t* positions,
                                  uint8_t* key_codes, uint8_t* val_codes, cudaStream_t stream);
+// cvq_attend with its two workspace parts given separately: the split partial states
+// (cvq_partials_bytes, 16-byte aligned) and one int32 arrival counter per (sequence, query
+// head), which must be zero when the kernel starts.  clear_counters > 0: once every
+// argument has passed its checks, first clear that many counters with an asynchronous
+// memset on `stream` (api.cu).
+cvq_status attend_into(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,
+                       int64_t key_cb_head_stride, const uint8_t* key_codes,
+                       const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
+                       int64_t val_cb_head_stride, int n_splits, float* partials, int* counters,
+                       float* out, float* lse, void* stream, size_t clear_counters);
 cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
                            const float* part_m, const float* part_l, float* out, float* lse,
                            cudaStream_t stream);

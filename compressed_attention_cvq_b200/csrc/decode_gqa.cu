@@ -29,8 +29,9 @@
 //     touch 32 different banks and never the same address.
 //
 // Tokens: kSlots = 4 per warp per step; slot sigma handles t_begin + sigma + kSlots*j.
-// The phase of a lane's 4 pairs starts from the exact fixed-point turn and advances by
-// e^{i theta_j kSlots} per step (rounding error ~1e-7 per step).  Code bytes of the
+// The phase of a lane's 4 pairs is re-seeded from the exact fixed-point turn at the start
+// of every tile and advances by e^{i theta_j kSlots} per step within it (at most
+// kSteps - 1 products, rounding error ~1e-7 each).  Code bytes of the
 // next tile are copied to shared memory with cp.async while the current tile computes.
 #include <cooperative_groups.h>
 
@@ -194,13 +195,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
                              load_q(a.q, a.q_dtype, qb + 2 * pp + 1) * qscale);
     }
   }
+  // phase of the lane's pairs: re-seeded from the exact turn at the first token of every
+  // tile, advanced by e^{i theta kSlots} per step within the tile (<= kSteps - 1 products)
   float2 ph[4], adv[4];
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int pp = p ^ (2 * fk);
-    ph[p] = phase_at(a.phase.F[4 * G + pp], t_begin + sigma);
-    adv[p] = phase_at(a.phase.F[4 * G + pp], C::kSlots);
-  }
+  for (int p = 0; p < 4; ++p) adv[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], C::kSlots);
   float* peer_xchg = cluster.map_shared_rank(xchg, rank ^ 1);
 
   float m_ref = -INFINITY;      // reference max (log2 units) of head hk; equal in all lanes
@@ -267,6 +266,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     float* xb = xchg + buf * (kTile * kHeads);
     float* pxb = peer_xchg + buf * (kTile * kHeads);
 
+#pragma unroll
+    for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
     float s_part[C::kSteps];
 #pragma unroll
     for (int st = 0; st < C::kSteps; ++st) {

@@ -7,6 +7,13 @@
 // hands it no allocator, or a decode loop that cannot pay for cudaMalloc's implicit
 // synchronization.  They pass only inputs and outputs; the intermediate partial states
 // go to g_static_scratch, which every GPU that loads this library holds until exit.
+//
+// Layout of the array (fixed, whatever the shape of a call):
+//   [0, kCounterBytes)              arrival counters, one int32 per (sequence, query head);
+//                                   no call ever writes partial states here
+//   [kCounterBytes, kScratchBytes)  split partial states of the current call
+// The counters a call uses are cleared on the call's stream before its decode kernel, so
+// a call never depends on what an earlier call (of any shape) left in the array.
 #include <mutex>
 
 #include "common.cuh"
@@ -15,20 +22,24 @@ using namespace cvq;
 
 namespace {
 
-constexpr size_t kStaticScratchFloats = CVQ_STATIC_SCRATCH_BYTES / sizeof(float);
-static_assert(CVQ_STATIC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte alignment");
+constexpr size_t kScratchBytes = CVQ_STATIC_SCRATCH_BYTES;
+constexpr size_t kCounterBytes = CVQ_STATIC_COUNTER_BYTES;
+constexpr size_t kCounterInts = kCounterBytes / sizeof(int);
+static_assert(kScratchBytes % 256 == 0 && kCounterBytes % 256 == 0,
+              "both regions keep 256-byte alignment");
+static_assert(kCounterBytes < kScratchBytes, "the partial states need room after the counters");
 
-// The partial states of the most recent call.  In host code this name is only a
-// stand-in for the symbol: its device address comes from cudaGetSymbolAddress.
-__device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
+// Counters, then the partial states of the most recent call.  In host code this name is
+// only a stand-in for the symbol: its device address comes from cudaGetSymbolAddress.
+__device__ __align__(256) unsigned char g_static_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 128;
-float* g_scratch_addr[kMaxDevices] = {};
+unsigned char* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
 // Device address of g_static_scratch on the current device, looked up once per device
 // (with that device current) and cached.
-cudaError_t scratch_address(float** out) {
+cudaError_t scratch_address(unsigned char** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -38,7 +49,7 @@ cudaError_t scratch_address(float** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<float*>(p);
+    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;
@@ -58,17 +69,22 @@ extern "C" CVQ_API cvq_status cvq_attend_static(
   if (s == nullptr) return CVQ_ERR_NULL;
   if (n_splits < 1 || n_splits > 4096) return CVQ_ERR_WORKSPACE;
   if (s->batch < 1 || s->n_q_heads < 1) return CVQ_ERR_SHAPE;
-  const size_t need = cvq_attend_workspace_bytes(s, n_splits);
-  if (need == 0)   // an invalid shape: cvq_attend reports which check fails, before any launch
+  const size_t parts = cvq_partials_bytes(s, n_splits);
+  if (parts == 0)   // an invalid shape: cvq_attend reports which check fails, before any launch
     return cvq_attend(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes, seq_lens,
                       val_cb, val_cb_head_stride, n_splits, nullptr, out, lse, stream);
-  if (need > CVQ_STATIC_SCRATCH_BYTES) return CVQ_ERR_STATIC_LIMIT;
+  const size_t n_counters = static_cast<size_t>(s->batch) * s->n_q_heads;
+  if (parts > kScratchBytes - kCounterBytes || n_counters > kCounterInts) return CVQ_ERR_STATIC_LIMIT;
 
-  float* base = nullptr;
+  unsigned char* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return CVQ_ERR_CUDA;
-  // The array is cvq_attend's workspace: the split partial states, then one arrival
-  // counter per (sequence, head).  Static device memory starts zeroed and every call
-  // leaves the counters zero, so nothing needs clearing.
-  return cvq_attend(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes, seq_lens,
-                    val_cb, val_cb_head_stride, n_splits, base, out, lse, stream);
+  int* counters = reinterpret_cast<int*>(base);
+  float* partials = reinterpret_cast<float*>(base + kCounterBytes);
+  // The arrival counters must start at zero.  A completed call leaves its counters zero,
+  // but the call clears them anyway (an asynchronous memset on its stream, after every
+  // argument check and before the decode kernel; it allocates nothing), so that it does not
+  // depend on any earlier call: one of another shape, or one whose kernel never completed.
+  return attend_into(s, q, q_dtype, key_cb, key_cb_head_stride, key_codes, val_codes, seq_lens,
+                     val_cb, val_cb_head_stride, n_splits, partials, counters, out, lse, stream,
+                     n_counters);
 }

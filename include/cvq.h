@@ -195,10 +195,14 @@ CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, in
  *   [B, Hq] as in cvq_combine.
  *   workspace  cvq_attend_workspace_bytes(shape, n_splits) bytes of device memory,
  *              16-byte aligned, owned by the caller: the split partial states followed
- *              by one int32 arrival counter per (sequence, head).  The counters must be
- *              zero before the first call (clear the workspace once after allocating
- *              it); every call leaves them zero.  Calls that share a workspace must be
- *              ordered on one stream.
+ *              by one int32 arrival counter per (sequence, head).  The counters sit
+ *              right after the partial states, so their offset depends on the shape
+ *              and n_splits.  They must be zero when a call starts: clear the
+ *              workspace after allocating it.  A call that completes leaves its own
+ *              counters zero, so later calls with the SAME shape and n_splits need no
+ *              clearing; before reusing a workspace with a different shape or n_splits,
+ *              clear it again (its counters would otherwise land on earlier partial
+ *              states).  Calls that share a workspace must be ordered on one stream.
  * ------------------------------------------------------------------------------- */
 CVQ_API size_t cvq_attend_workspace_bytes(const cvq_shape* shape, int n_splits);
 CVQ_API cvq_status cvq_attend(const cvq_shape* shape, const void* q, int q_dtype,
@@ -286,15 +290,22 @@ CVQ_API cvq_status cvq_encode_append(const cvq_shape* shape, const float* keys, 
  * synchronization.  The call itself allocates nothing.
  *
  *   Arguments as in cvq_decode_attn_gqa, then out [B, Hq, 128] and lse [B, Hq] as in
- *   cvq_combine.  cvq_attend_workspace_bytes(shape, n_splits) must fit in
- *   CVQ_STATIC_SCRATCH_BYTES (4 MiB, held by every GPU that loads the library until
- *   the process exits); larger calls return CVQ_ERR_STATIC_LIMIT before any launch.
+ *   cvq_combine.  The array (CVQ_STATIC_SCRATCH_BYTES = 4 MiB, held by every GPU that
+ *   loads the library until the process exits) has a fixed layout: its first
+ *   CVQ_STATIC_COUNTER_BYTES (32 KiB) hold the arrival counters, one int32 per
+ *   (sequence, query head), and the rest holds the split partial states.  So a call
+ *   fits when cvq_partials_bytes(shape, n_splits) <= 4 MiB - 32 KiB and
+ *   batch * n_q_heads <= 8192; any other call returns CVQ_ERR_STATIC_LIMIT before any
+ *   launch.  Every call first clears its counters (an asynchronous cudaMemsetAsync on
+ *   `stream`, issued after all argument checks; it allocates nothing), so calls of any
+ *   shape may follow one another in any order.
  *   The first call on a device looks up the array's device address with that device
  *   current (cudaGetSymbolAddress), so make that first call before any stream capture.
  *   Every call reuses the same array: calls whose work overlaps on the GPU (other
  *   streams, other host threads) race on it and must be serialized by the caller.
  * ------------------------------------------------------------------------------- */
 #define CVQ_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+#define CVQ_STATIC_COUNTER_BYTES (32u * 1024u)
 CVQ_API cvq_status cvq_attend_static(const cvq_shape* shape, const void* q, int q_dtype,
                                      const float* key_cb, int64_t key_cb_head_stride,
                                      const uint8_t* key_codes, const uint8_t* val_codes,

@@ -59,3 +59,19 @@ def test_encode_work_by_hand():
                                                    (4, 1000, 2.0, 4 * 1000 / 2e-3)])
 def test_whole_job_rate(world, units, ms, expect):
     assert math.isclose(bench.whole_job_rate(world, units, ms), expect, rel_tol=1e-12)
+
+
+def test_roofline_legs_by_hand():
+    # 128K layer, R = 1, 1965 MHz, 148 SMs:
+    #   FP32: 131072 x 32 x 272 FLOP / 2 = 570,425,344 FMA at 123.74 lanes/clk
+    #         -> 4,609,870.2 clk per SM-set -> / (148 x 1.965e9) = 15.851 us
+    #   SFU:  131072 x 64 sin+cos pairs at 7.95 + 131072 x 32 exp2 at 15.90 per clk
+    #         -> 1,055,173.0 + 263,791.1 = 1,318,964.2 clk -> 4.5353 us
+    #   HBM:  35,651,584 B at 6528.7 GB/s -> 5.4607 us
+    legs = bench.roofline_legs(W["llama8b_layer_T131072_R1"], 131072, 1965.0, 6528.7)
+    clk = 148 * 1965e6
+    assert math.isclose(legs["fp32_us"], 570_425_344 / 123.74 / clk * 1e6, rel_tol=1e-12)
+    assert math.isclose(legs["fp32_us"], 15.851, rel_tol=1e-4)
+    assert math.isclose(legs["sfu_us"], 4.5353, rel_tol=1e-4)
+    assert math.isclose(legs["hbm_us"], 35_651_584 / 6528.7e9 * 1e6, rel_tol=1e-12)
+    assert max(legs, key=legs.get) == "fp32_us"

@@ -84,3 +84,22 @@ def test_fused_full_size_128k():
     ref_out, ref_lse = run_oracle(d, heads=heads)
     assert_close(out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
                  ref_out, ref_lse, heads=heads)
+
+
+@pytest.mark.gpu
+def test_128k_layer_with_one_and_two_splits():
+    """The 128K-token layer decoded with 1 and 2 splits: each CTA pair walks 64K-128K
+    positions, 256 to 512 tiles, so the RoPE phase must stay exact over a long split (it is
+    re-seeded from the exact fixed-point turn at every tile and advanced within it)."""
+    w = workloads.WORKLOADS["llama8b_layer_T131072_R1"]
+    d = workloads.generate(w)
+    dd = to_device(d)
+    heads = [(0, 1), (0, 14), (0, 31)]
+    ref_out, ref_lse = run_oracle(d, heads=heads)
+    for n_splits in (1, 2):
+        out, lse = cvq.attend(dd["q"], dd["key_cb"], dd["val_cb"], dd["key_codes"],
+                              dd["val_codes"], dd["seq_lens"], d["rope_base"], n_splits=n_splits,
+                              form="gqa")
+        torch.cuda.synchronize()
+        assert_close(out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                     ref_out, ref_lse, heads=heads)
