@@ -480,7 +480,8 @@ def run_gpu(args):
         # timed steps, so that the clock sampler sees the kernel under load for many samples.
         # The steps (one per input set) are captured once in a CUDA graph and replayed, so
         # the host's enqueue cost does not gate short kernels.
-        sustained = sustained_run(step, args, n_sets, stream, dev)
+        sustained = (None if args.no_sustained
+                     else sustained_run(step, args, n_sets, stream, dev))
     if world > 1:
         dist.barrier()
     starts = [ev_start] + [e["end"] for e in evs[:-1]]
@@ -711,6 +712,8 @@ def main(argv=None):
     ap.add_argument("--append", action="store_true",
                     help="each step first encodes the step's new key/value into the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the sustained-load loop after the timed steps (profiling runs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

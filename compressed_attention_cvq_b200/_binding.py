@@ -10,7 +10,9 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libcvq.so")
+# CVQ_LIBRARY=debug loads the debug build (device-side range checks, libcvq_debug.so)
+LIB_PATH = os.path.join(PKG, "libcvq_debug.so" if os.environ.get("CVQ_LIBRARY") == "debug"
+                        else "libcvq.so")
 
 CVQ_OK = 0
 CVQ_F32 = 0
@@ -35,7 +37,7 @@ class cvq_shape(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libcvq.so not built at {LIB_PATH}; run "
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run "
                           "`python -m compressed_attention_cvq_b200.build` (needs nvcc)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
@@ -88,6 +90,15 @@ EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partia
             "cvq_encode_append", "cvq_attend_workspace_bytes", "cvq_attend",
             "cvq_fault_status"]
 CVQ_FAULT_COPY_TIMEOUT = 1
+CVQ_FAULT_BOUNDS = 2
+FAULT_NAMES = {CVQ_FAULT_COPY_TIMEOUT: "copy_timeout", CVQ_FAULT_BOUNDS: "bounds"}
+
+
+def fault_names(word: int) -> list:
+    """Names of the bits set in a device fault word (cvq_fault_status); unknown bits as hex."""
+    names = [n for bit, n in sorted(FAULT_NAMES.items()) if word & bit]
+    rest = word & ~sum(FAULT_NAMES)
+    return names + ([hex(rest)] if rest else [])
 
 
 def status_str(st: int) -> str:

@@ -2,10 +2,14 @@
 
     python -m compressed_attention_cvq_b200.build          # build (incremental)
     python -m compressed_attention_cvq_b200.build --force  # rebuild everything
+    python -m compressed_attention_cvq_b200.build --debug-bounds   # also the debug build
 
 Each csrc/*.cu is compiled to an object under _build/ (skipped when the object is
 newer than the source and the headers), then all objects are linked into
-compressed_attention_cvq_b200/libcvq.so.
+compressed_attention_cvq_b200/libcvq.so.  The debug build compiles the same sources with
+-DCVQ_DEBUG_BOUNDS (device-side range checks that set CVQ_FAULT_BOUNDS in the fault word
+and skip the access) into _build_debug/ and compressed_attention_cvq_b200/libcvq_debug.so,
+which the binding loads when CVQ_LIBRARY=debug.
 """
 from __future__ import annotations
 
@@ -23,6 +27,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libcvq.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libcvq_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -47,14 +53,16 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(p) > t for p in [src, *_deps()])
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          debug_bounds: bool = False) -> str:
+    build_dir, lib_path = (BUILD_DEBUG, LIB_DEBUG) if debug_bounds else (BUILD, LIB)
+    extra = list(extra or []) + (["-DCVQ_DEBUG_BOUNDS"] if debug_bounds else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     cc = nvcc()
-    extra = list(extra or [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if force or _stale(obj, src):
             cmd = [cc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
             if verbose:
@@ -68,14 +76,15 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
 
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs, "-lpthread", "-ldl", "-lrt"]
+    if (force or not os.path.exists(lib_path)
+            or any(os.path.getmtime(o) > os.path.getmtime(lib_path) for o in objs)):
+        cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", lib_path, *objs, "-lpthread", "-ldl", "-lrt"]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib_path
 
 
 def main(argv=None):
@@ -83,10 +92,14 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print register / smem usage")
+    ap.add_argument("--debug-bounds", action="store_true",
+                    help="also build libcvq_debug.so with device-side range checks")
     args = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if args.ptxas_info else []
     lib = build(force=args.force or args.ptxas_info, verbose=args.verbose or args.ptxas_info, extra=extra)
     print(lib)
+    if args.debug_bounds:
+        print(build(force=args.force, verbose=args.verbose, debug_bounds=True))
 
 
 if __name__ == "__main__":

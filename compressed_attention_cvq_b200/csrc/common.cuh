@@ -62,6 +62,13 @@ __device__ __forceinline__ float2 phase_at(unsigned long long F, int t) {
   return phase_from_turn(F * static_cast<unsigned long long>(static_cast<unsigned>(t)));
 }
 
+// Order-preserving map of a float (not NaN) to an int and back, for integer atomicMax.
+__device__ __forceinline__ int ord_of(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float float_of_ord(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
@@ -115,13 +122,31 @@ struct DecodeArgs {
 
 // ---- bits of the device fault word (cvq_fault_status) ----
 constexpr unsigned int kFaultCopyTimeout = CVQ_FAULT_COPY_TIMEOUT;   // a TMA copy did not land in time
+constexpr unsigned int kFaultBounds = CVQ_FAULT_BOUNDS;             // a debug range check failed
+
+// Range check of the debug build (compiled with -DCVQ_DEBUG_BOUNDS): true if i < n;
+// otherwise it sets kFaultBounds in the fault word and returns false, and the caller skips
+// the access (a load yields 0) and runs on, so that every barrier is still met.  It never
+// traps.  In the regular build it is always true and compiles away.
+__device__ __forceinline__ bool in_bounds(unsigned int* fault, size_t i, size_t n) {
+#ifdef CVQ_DEBUG_BOUNDS
+  if (i < n) return true;
+  atomicOr(fault, kFaultBounds);
+  return false;
+#else
+  (void)fault; (void)i; (void)n;
+  return true;
+#endif
+}
 
 constexpr int kCodeBoxRows = 32;   // codes per TMA box of the codebook maps
 
 // ---- mbarrier + TMA (bulk copy engine) helpers ----
-// A bounded wait polls the barrier (try_wait, no suspend hint) and gives up once this many
-// nanoseconds of %globaltimer have passed since its first poll.
+// A bounded wait polls the barrier with try_wait, which may suspend the thread until the
+// phase completes or for about kMbarSuspendHintNs, and gives up once kMbarWaitLimitNs of
+// %globaltimer have passed since its first poll.
 constexpr unsigned long long kMbarWaitLimitNs = 2000000000ull;   // 2 s
+constexpr unsigned int kMbarSuspendHintNs = 100000u;              // 100 us per poll at most
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -142,10 +167,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned int parity) {
   for (int i = 0;; ++i) {
     uint32_t done;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(done)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kMbarSuspendHintNs)
         : "memory");
     if (done) return true;
     unsigned long long now;
@@ -193,10 +218,12 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
                                            int n_heads, int expected) {
   static_assert(W == 1 || W == 2 || W == 4, "warps per head");
   constexpr int D = 4 / W;                         // output dims per lane
-  int* ctr = a.counters + static_cast<size_t>(b) * gridDim.y + unit;
+  const size_t ctr_i = static_cast<size_t>(b) * gridDim.y + unit;
+  const bool ctr_ok = in_bounds(a.fault, ctr_i, static_cast<size_t>(a.batch) * a.n_q_heads);
+  int* ctr = a.counters + (ctr_ok ? ctr_i : 0);
   int old = 0;
   __syncthreads();                       // this CTA's partial states are all written
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && ctr_ok) {
     // release: the CTA's partials (ordered before this by the barrier) are visible at GPU
     // scope before the count; acquire: the last CTA then sees every other CTA's partials
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
@@ -208,6 +235,7 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
   const int wl = warp % W;
   for (int hh = warp / W; hh < n_heads; hh += (blockDim.x >> 5) / W) {
     const size_t row = static_cast<size_t>(b) * a.n_q_heads + hq0 + hh;
+    if (!in_bounds(a.fault, row, static_cast<size_t>(a.batch) * a.n_q_heads)) continue;
     const float* pm = a.part_m + row * S;
     const float* pl = a.part_l + row * S;
     const float* po = a.part_o + row * S * kHeadDim + 32 * wl + lane;
@@ -264,7 +292,7 @@ __device__ __forceinline__ void merge_tail(const DecodeArgs& a, int b, int unit,
     for (int j = 0; j < D; ++j) orow[32 * W * j] = acc[j] / L;
     if (wl == 0 && lane == 0) a.lse[row] = M + logf(L);
   }
-  if (threadIdx.x == 0) atomicExch(ctr, 0);
+  if (threadIdx.x == 0 && ctr_ok) atomicExch(ctr, 0);
 }
 
 // Launchers (defined next to their kernels).  Return cudaSuccess or the launch error.

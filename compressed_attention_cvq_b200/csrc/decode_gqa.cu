@@ -62,7 +62,7 @@ struct Cfg {
   static constexpr int kXchg = 2 * kTile * kHeads;                    // floats (2 buffers)
   static constexpr int kCodeBytes = 2 * kTile * R * 16;               // 2 buffers x (key 8 B + val 8 B) x R
   static constexpr size_t kSmem = sizeof(float4) * kCodeChunks +
-                                  sizeof(float) * (kBins + kXchg + kWarps * kHeads + 2 * kHeads) +
+                                  sizeof(float) * (kBins + kXchg + kWarps * kHeads + 4 * kHeads) +
                                   kCodeBytes + 16;   // + the TMA mbarrier
   static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
 };
@@ -109,9 +109,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   float* bins = reinterpret_cast<float*>(smem4 + C::kCodeChunks);     // [R][256][4][8]
   float* xchg = bins + C::kBins;                                      // [2][kTile][4]
   float* red = xchg + C::kXchg;                                       // [kWarps][4]
-  float* fh = red + C::kWarps * kHeads;                               // [4] tile max / factors
-  float* mtile = fh + kHeads;                                         // [4]
-  uint8_t* code_s = reinterpret_cast<uint8_t*>(mtile + kHeads);       // [2][kTile][R][key 8 | val 8]
+  float* fh = red + C::kWarps * kHeads;                               // [4] rescale factors
+  int* mslot = reinterpret_cast<int*>(fh + kHeads);                   // [3][4] tile maxima (ord)
+  uint8_t* code_s = reinterpret_cast<uint8_t*>(mslot + 3 * kHeads);   // [2][kTile][R][key 8 | val 8]
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(code_s + C::kCodeBytes);   // codebook copies
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -134,13 +134,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   const int t_begin = split * a.split_tokens;
   const int t_end = min(t_begin + a.split_tokens, L);
   const size_t part_row = (static_cast<size_t>(b) * a.n_q_heads + hq0) * a.n_splits + split;
+  // the last partial-state row this CTA writes lies inside the partial states
+  const bool parts_ok = in_bounds(a.fault, part_row + static_cast<size_t>(kHeads - 1) * a.n_splits,
+                                  static_cast<size_t>(a.batch) * a.n_q_heads * a.n_splits);
 
   if (t_begin >= t_end) {   // both CTAs of the pair take this branch together
-    for (int i = tid; i < kHeads * 64; i += C::kThreads) {
+    for (int i = tid; i < kHeads * 64 && parts_ok; i += C::kThreads) {
       const int hh = i >> 6, d = i & 63;
       a.part_o[(part_row + static_cast<size_t>(hh) * a.n_splits) * kHeadDim + rank * 64 + d] = 0.f;
     }
-    if (rank == 0 && tid < kHeads) {
+    if (rank == 0 && tid < kHeads && parts_ok) {
       a.part_m[part_row + static_cast<size_t>(tid) * a.n_splits] = -INFINITY;
       a.part_l[part_row + static_cast<size_t>(tid) * a.n_splits] = 0.f;
     }
@@ -154,7 +157,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     for (int i = tid; i < kTile * R; i += C::kThreads) {
       const int tt = i % kTile, r = i / kTile;
       const int t = t_tile + tt;
-      if (t < t_end) {
+      if (t < t_end && in_bounds(a.fault, t, a.t_cap) &&
+          in_bounds(a.fault, ((buf * kTile + tt) * R + r) * 16 + 15, C::kCodeBytes)) {
         const size_t off = (code_row + t) * (16 * R) + r * 16 + rank * 8;
         uint8_t* dst = code_s + ((buf * kTile + tt) * R + r) * 16;
         cp_async8(dst, a.key_codes + off);
@@ -174,6 +178,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   stage_codes(t_begin, 0);
   for (int i = tid; i < C::kBins / 4; i += C::kThreads)
     reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid < 3 * kHeads) mslot[tid] = ord_of(-INFINITY);
 
   // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2
   // units.  Slot j holds head (k ^ j) & 3: with this lane-dependent order the butterfly
@@ -224,17 +229,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   // 81.8 -> 80.9 us, 128K R = 1 +0.5-1 us).
   constexpr bool kEarlyValueCopy = C::kMinBlocks == 1;
 
-  // Software pipeline over tiles.  Iteration t: key side of tile t -> arrive on the
-  // cluster barrier -> bin atomics of tile t-1 (weights and value codes kept in
-  // registers) -> wait on the barrier -> scores, max and weights of tile t.  The
-  // atomics overlap the exchange with the peer CTA.
-  float w[C::kSteps];            // weights of the previous tile's tokens (head hk)
+  // Software pipeline over tiles.  Iteration t: key side of tile t -> cluster barrier (the
+  // peer's partial scores of tile t have arrived; every warp's tile t-1 maximum is in
+  // mslot) -> full scores and the warp's maxima of tile t into mslot -> raise the reference
+  // max from tile t-1's maximum if needed -> weights and bin atomics of tile t-1 (scores and
+  // value codes kept in registers for one iteration).  The only barrier of a tile is the
+  // cluster barrier (plus the code-copy barrier at its start); no CTA-wide max reduction.
+  float sp[C::kSteps];           // scores of the previous tile's tokens (head hk; -inf = none)
   uint32_t vw[C::kSteps][R];     // value code bytes of those tokens (groups 4 gh .. 4 gh + 3)
-  bool prev_valid[C::kSteps];
 #pragma unroll
   for (int st = 0; st < C::kSteps; ++st) {
-    prev_valid[st] = false;
-    w[st] = 0.f;
+    sp[st] = -INFINITY;
 #pragma unroll
     for (int r = 0; r < R; ++r) vw[st][r] = 0u;
   }
@@ -242,25 +247,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   auto bin_atomics = [&]() {
 #pragma unroll
     for (int st = 0; st < C::kSteps; ++st) {
+      float e;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(sp[st] - m_ref));   // -inf -> 0
+      l_acc += (gh == 0) ? e : 0.f;     // lanes k and k ^ 4 hold the same head
       // R = 1 skips the per-token branch: a token past the split end has weight 0 (score
       // -inf), so its atomics add 0 to some bin (measured: faster at R = 1, slower at R = 2)
-      if (R == 1 || prev_valid[st]) {
+      if (R == 1 || sp[st] != -INFINITY) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           const uint32_t rot = __funnelshift_r(vw[st][r], vw[st][r], 8 * tau);  // byte i: group 4gh + ((i + tau) & 3)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int c = static_cast<int>(__byte_perm(rot, 0u, 0x4440u + i));
-            atomicAdd(bins + r * (kCodes * kHeads * kLocalGroups) + c * (kHeads * kLocalGroups) + bin_off[i],
-                      w[st]);
+            const int bi = r * (kCodes * kHeads * kLocalGroups) + c * (kHeads * kLocalGroups) + bin_off[i];
+            if (in_bounds(a.fault, bi, C::kBins)) atomicAdd(bins + bi, e);
           }
         }
       }
     }
   };
 
+  // Raise the reference max of head hk to the maximum mt of a finished tile when mt exceeds
+  // it by more than the slack, rescaling bins and l.  Every warp reads the same mt values
+  // (lanes cover all 4 heads), so the branch is uniform over the CTA, and both CTAs of the
+  // pair hold bit-identical scores, so they decide alike.  The caller guarantees that every
+  // atomic already issued has completed (a CTA-wide barrier since) and that none of the
+  // tile's own atomics has started.
+  auto raise_ref = [&](float mt) {
+    const bool raise = (m_ref == -INFINITY && mt != -INFINITY) || (mt > m_ref + kRescaleSlack);
+    if (__any_sync(0xffffffffu, raise)) {
+      const float m_new = raise ? mt : m_ref;
+      const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
+      // bins hold nothing before the first raise of every head: rescale only once some
+      // head had a finite reference
+      const bool rescale = __any_sync(0xffffffffu, m_ref != -INFINITY);
+      l_acc *= f;
+      m_ref = m_new;
+      if (rescale) {
+        if (tid < kHeads) fh[tid] = f;       // thread tid < 4 is lane tid: head tid
+        __syncthreads();
+        for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] *= fh[(i >> 3) & 3];
+        __syncthreads();
+      }
+    }
+  };
+
   // one tile: FULL = every token of the tile is inside the split (no per-token checks)
-  auto run_tile = [&](const int t_tile, const int buf, auto full_tag, const bool last) {
+  auto run_tile = [&](const int t_tile, const int tile, const int buf, auto full_tag, const bool last) {
     constexpr bool FULL = decltype(full_tag)::value;
     const uint8_t* cb = code_s + static_cast<size_t>(buf) * kTile * R * 16;
     float* xb = xchg + buf * (kTile * kHeads);
@@ -269,48 +302,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 #pragma unroll
     for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
     float s_part[C::kSteps];
+    constexpr int kGS = C::kSteps >= 4 ? 4 : C::kSteps;   // steps per pass group
 #pragma unroll
-    for (int st = 0; st < C::kSteps; ++st) {
-      const int tt = st * C::kSlots + sigma;             // token within the tile
-      float2 kw[4];
+    for (int sg = 0; sg < C::kSteps; sg += kGS) {
+      float pv[kGS][kHeads];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int c = cb[(tt * R + r) * 16 + k];
-        // chunk fk first: lanes 0-3 and 4-7 of a token then hit 8 distinct bank quads;
-        // lo holds the lane's slots 0, 1 and hi its slots 2, 3 (pairs 2 fk, ... see qv)
-        const float4* src = cw_s + ((r * kCodes + c) * kLocalGroups + k) * 2;
-        const float4 lo = src[fk], hi = src[fk ^ 1];
-        if (r == 0) {
-          kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
-          kw[2] = make_float2(hi.x, hi.y); kw[3] = make_float2(hi.z, hi.w);
-        } else {
-          kw[0] = __fadd2_rn(kw[0], make_float2(lo.x, lo.y));
-          kw[1] = __fadd2_rn(kw[1], make_float2(lo.z, lo.w));
-          kw[2] = __fadd2_rn(kw[2], make_float2(hi.x, hi.y));
-          kw[3] = __fadd2_rn(kw[3], make_float2(hi.z, hi.w));
+      for (int u = 0; u < kGS; ++u) {
+        const int tt = (sg + u) * C::kSlots + sigma;
+        float2 kw[4];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int c = cb[(tt * R + r) * 16 + k];
+          const int ci = ((r * kCodes + c) * kLocalGroups + k) * 2;
+          const float4* src = cw_s + (in_bounds(a.fault, ci + 1, C::kCodeChunks) ? ci : 0);
+          const float4 lo = src[fk], hi = src[fk ^ 1];
+          if (r == 0) {
+            kw[0] = make_float2(lo.x, lo.y); kw[1] = make_float2(lo.z, lo.w);
+            kw[2] = make_float2(hi.x, hi.y); kw[3] = make_float2(hi.z, hi.w);
+          } else {
+            kw[0] = __fadd2_rn(kw[0], make_float2(lo.x, lo.y));
+            kw[1] = __fadd2_rn(kw[1], make_float2(lo.z, lo.w));
+            kw[2] = __fadd2_rn(kw[2], make_float2(hi.x, hi.y));
+            kw[3] = __fadd2_rn(kw[3], make_float2(hi.z, hi.w));
+          }
         }
-      }
-      float2 part2[kHeads];
+        float2 part2[kHeads];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 x = cmul(ph[p], kw[p]);
+        for (int p = 0; p < 4; ++p) {
+          const float2 x = cmul(ph[p], kw[p]);
 #pragma unroll
-        for (int j = 0; j < kHeads; ++j)
-          part2[j] = p == 0 ? __fmul2_rn(qv[j][p], x) : __ffma2_rn(qv[j][p], x, part2[j]);
-        ph[p] = cmul(ph[p], adv[p]);
+          for (int j = 0; j < kHeads; ++j)
+            part2[j] = p == 0 ? __fmul2_rn(qv[j][p], x) : __ffma2_rn(qv[j][p], x, part2[j]);
+          ph[p] = cmul(ph[p], adv[p]);
+        }
+#pragma unroll
+        for (int j = 0; j < kHeads; ++j) pv[u][j] = part2[j].x + part2[j].y;
       }
-      // butterfly over the token's 8 lanes (slot j of lane k is head (k ^ j) & 3)
-      const float p0 = part2[0].x + part2[0].y, p1 = part2[1].x + part2[1].y;
-      const float p2 = part2[2].x + part2[2].y, p3 = part2[3].x + part2[3].y;
-      const float r0 = p0 + __shfl_xor_sync(0xffffffffu, p2, 2);
-      const float r1 = p1 + __shfl_xor_sync(0xffffffffu, p3, 2);
-      float v = r0 + __shfl_xor_sync(0xffffffffu, r1, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      s_part[st] = v;
-      if (k < 4) pxb[tt * kHeads + hk] = v;
+#pragma unroll
+      for (int u = 0; u < kGS; ++u) {
+        const int tt = (sg + u) * C::kSlots + sigma;
+        const float r0 = pv[u][0] + __shfl_xor_sync(0xffffffffu, pv[u][2], 2);
+        const float r1 = pv[u][1] + __shfl_xor_sync(0xffffffffu, pv[u][3], 2);
+        float v = r0 + __shfl_xor_sync(0xffffffffu, r1, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        s_part[sg + u] = v;
+        if (k < 4 && in_bounds(a.fault, tt * kHeads + hk, kTile * kHeads)) pxb[tt * kHeads + hk] = v;
+      }
     }
     cluster_arrive_release();
-    bin_atomics();                      // previous tile, while the exchange completes
     cluster_wait_acquire();             // the peer's partials of this tile are in xb
     if (kEarlyValueCopy && last && warp == 0) {
       // every thread of the CTA is past its last key gather: bring in the value codewords
@@ -321,50 +360,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     }
 
     // full scores (the same order of addition in both CTAs -> identical values)
-    float s[C::kSteps];
+    float sc[C::kSteps];
+    uint32_t vn[C::kSteps][R];
     float mx = -INFINITY;
 #pragma unroll
     for (int st = 0; st < C::kSteps; ++st) {
       const int tt = st * C::kSlots + sigma;
       const float other = xb[tt * kHeads + hk];
       const float v = rank == 0 ? s_part[st] + other : other + s_part[st];
-      s[st] = (FULL || t_tile + tt < t_end) ? v : -INFINITY;
-      mx = fmaxf(mx, s[st]);
-      prev_valid[st] = FULL || t_tile + tt < t_end;
+      sc[st] = (FULL || t_tile + tt < t_end) ? v : -INFINITY;
+      mx = fmaxf(mx, sc[st]);
 #pragma unroll
       for (int r = 0; r < R; ++r)
-        vw[st][r] = *reinterpret_cast<const uint32_t*>(cb + (tt * R + r) * 16 + 8 + 4 * gh);
+        vn[st][r] = *reinterpret_cast<const uint32_t*>(cb + (tt * R + r) * 16 + 8 + 4 * gh);
     }
-    // CTA-wide max per head: one barrier, then every warp reduces all warps' maxima
+    // this warp's maximum per head into the tile's slot (lanes 0..3: heads 0..3); the
+    // slot two tiles back, read by every warp before this tile's cluster barrier, is reset
+    // for the next tile
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (lane < kHeads) red[warp * kHeads + lane] = mx;
-    __syncthreads();
-    float mt = red[lane];                                   // entry lane: head lane & 3
-#pragma unroll
-    for (int e = 32; e < C::kWarps * kHeads; e += 32) mt = fmaxf(mt, red[e + lane]);
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));   // lane l: tile max of head l & 3 = hk
-    const bool raise = (m_ref == -INFINITY) || (mt > m_ref + kRescaleSlack);
-    if (__any_sync(0xffffffffu, raise)) {   // the same decision in every warp of the CTA
-      const float m_new = raise ? mt : m_ref;
-      const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
-      l_acc *= f;
-      m_ref = m_new;
-      if (tid < kHeads) fh[tid] = f;       // thread tid < 4 is lane tid: head tid
-      __syncthreads();                     // every atomic of the previous tile is done
-      for (int i = tid; i < C::kBins; i += C::kThreads) bins[i] *= fh[(i >> 3) & 3];
-      __syncthreads();
+    if (lane < kHeads) atomicMax(mslot + (tile % 3) * kHeads + lane, ord_of(mx));
+    if (tid < kHeads) mslot[((tile + 1) % 3) * kHeads + tid] = ord_of(-INFINITY);
+    if (tile > 0) {
+      // every warp's maximum of the previous tile landed before this tile's cluster
+      // barrier, and so did every atomic issued before it
+      raise_ref(float_of_ord(mslot[((tile + 2) % 3) * kHeads + hk]));
+      bin_atomics();                    // previous tile
     }
-    // weights of this tile (0 for tokens past the end); lanes k and k ^ 4 hold the same
-    // head, so only k < 4 adds to l
 #pragma unroll
     for (int st = 0; st < C::kSteps; ++st) {
-      float e;
-      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(s[st] - m_ref));
-      w[st] = e;
-      l_acc += (gh == 0) ? e : 0.f;
+      sp[st] = sc[st];
+#pragma unroll
+      for (int r = 0; r < R; ++r) vw[st][r] = vn[st][r];
     }
   };
 
@@ -377,12 +405,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     }
     if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
     if (t_tile + kTile <= t_end) {
-      run_tile(t_tile, buf, std::integral_constant<bool, true>(), tile + 1 == n_tiles);
+      run_tile(t_tile, tile, buf, std::integral_constant<bool, true>(), tile + 1 == n_tiles);
     } else {
-      run_tile(t_tile, buf, std::integral_constant<bool, false>(), tile + 1 == n_tiles);
+      run_tile(t_tile, tile, buf, std::integral_constant<bool, false>(), tile + 1 == n_tiles);
     }
   }
-  bin_atomics();                // the last tile
+  // the last tile: its maxima are complete once every warp is past its scores
+  __syncthreads();
+  raise_ref(float_of_ord(mslot[((n_tiles - 1) % 3) * kHeads + hk]));
+  bin_atomics();
 
   // ---- l: lanes hold disjoint shares of head hk; sum over slots, halves and warps ----
   l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 4);
@@ -391,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   __syncthreads();                                   // every bin update is done
   if (lane < kHeads) red[warp * kHeads + lane] = l_acc;
   __syncthreads();
-  if (rank == 0 && tid < kHeads) {
+  if (rank == 0 && tid < kHeads && parts_ok) {
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w) v += red[w * kHeads + tid];
@@ -431,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 #pragma unroll
     for (int d = 0; d < 8; ++d) part_s[(warp * 32 + lane) * 8 + d] = acc[d ^ (4 * fv)];
     __syncthreads();
-    for (int o = tid; o < kHeads * kLocalGroups * 8; o += C::kThreads) {
+    for (int o = tid; o < kHeads * kLocalGroups * 8 && parts_ok; o += C::kThreads) {
       const int d = o & 7, ln = o >> 3;                // ln = head * 8 + local group
       float v = 0.f;
 #pragma unroll

@@ -189,7 +189,8 @@ __global__ void __launch_bounds__(kSimpleThreads) decode_simple_kernel(const Dec
           for (int gi = 0; gi < kGroups / TPT; ++gi) {
             const int G = TPT == 1 ? gi : 4 * part + gi;
             const int c = TPT == 1 ? code_byte(vc[r], gi) : static_cast<int>((vword >> (8 * gi)) & 255u);
-            atomicAdd(bh + (G * R + r) * kCodes + c, w);
+            if (in_bounds(a.fault, (G * R + r) * kCodes + c, kGroups * R * kCodes))
+              atomicAdd(bh + (G * R + r) * kCodes + c, w);
           }
         }
       }

@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
       const int r = (i / (kWTile / 16)) % rc;
       const int q16 = i % (kWTile / 16);
       const int t = t_tile + 16 * q16;
-      if (t < t_end) {
+      if (t < t_end && in_bounds(a.fault, t + 15, a.t_cap)) {
         const uint8_t* src = (kind ? a.val_codes : a.key_codes) + (code_row0 + r) * a.t_cap + t;
         cp_async16(code_s + ((buf * 2 + kind) * kRC + r) * kWTile + 16 * q16, src);
       }
@@ -282,8 +282,10 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     float sA = 0.f, sB = 0.f;
     for (int q = 0; q < C; ++q) {
       const float* px = cluster.map_shared_rank(xo, q);
-      sA += px[tA * kWHeads + hh];
-      sB += px[tB * kWHeads + hh];
+      if (in_bounds(a.fault, tB * kWHeads + hh, kWTile * kWHeads)) {
+        sA += px[tA * kWHeads + hh];
+        sB += px[tB * kWHeads + hh];
+      }
     }
     if (t_tile + tA >= t_end) sA = -INFINITY;
     if (t_tile + tB >= t_end) sB = -INFINITY;
@@ -334,7 +336,8 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
         if (i < rc) {
           const uint32_t wd = r < 4 ? v4.x : (r < 8 ? v4.y : v4.z);
           const int c = (wd >> (8 * (r & 3))) & (kWideCodes - 1);
-          atomicAdd(&bins[c * kBinStride + 4 * r + hh], wt);
+          if (in_bounds(a.fault, c * kBinStride + 4 * r + hh, kWideCodes * kBinStride))
+            atomicAdd(&bins[c * kBinStride + 4 * r + hh], wt);
           r = (r + 1 == rc) ? 0 : r + 1;
         }
       }

@@ -1,6 +1,6 @@
 """Run the unit-throughput probes on GPU 0 and print one JSON object.
 
-    python -m compressed_attention_cvq_b200.microbench
+    python -m compressed_attention_cvq_b200.microbench [kind ...]   # all probes, or only these
 
 Builds microbench/libcvq_micro.so on first use (nvcc, sm_100a).  For each probe:
 operations per second and per SM per clock at the median SM clock sampled while it
@@ -19,8 +19,13 @@ KINDS = {0: "ffma", 1: "ffma2 (f32x2, 2 FMA each)", 2: "sincos (__sincosf)", 3: 
          7: "atomicAdd f32 random", 8: "atomicAdd f32 same address", 9: "shfl_xor",
          10: "red.shared.add.f32 distinct", 11: "red.shared.add.u32 distinct",
          12: "red.shared.add.u64 distinct", 13: "plain f32 ld/add/st distinct",
-         14: "plain float4 ld/add/st conflict-free", 15: "mixed: lds128 + 2 x red.f32"}
-ITERS = {0: 4000, 1: 2000, 2: 1000, 3: 1000, 4: 4000, 5: 4000, 6: 2000, 7: 2000, 8: 500, 9: 2000, 10: 2000, 11: 2000, 12: 2000, 13: 2000, 14: 2000, 15: 2000}
+         14: "plain float4 ld/add/st conflict-free", 15: "mixed: lds128 + 2 x red.f32",
+         16: "red.global.add.v4.f32 random (L2, 64 KB per CTA)",
+         17: "red.global.add.f32 random (L2, 64 KB per CTA)",
+         18: "red.global.add.v4.f32, 25% on 4 hot slots"}
+ITERS = {0: 4000, 1: 2000, 2: 1000, 3: 1000, 4: 4000, 5: 4000, 6: 2000, 7: 2000, 8: 500, 9: 2000, 10: 2000, 11: 2000, 12: 2000, 13: 2000, 14: 2000, 15: 2000,
+         16: 200, 17: 200, 18: 100}
+GLOBAL_KINDS = (16, 17, 18)     # take a scratch buffer of blocks x 16384 floats
 
 
 def build():
@@ -49,15 +54,24 @@ def main():
                             "--format=csv,noheader,nounits", "-lms", "100"],
                            stdout=subprocess.PIPE, text=True)
     rows = {}
+    scratch = None
+    only = [int(k) for k in sys.argv[1:]]
     for kind, name in KINDS.items():
+        if only and kind not in only:
+            continue
         blocks, threads = sms * 4, 256
+        dst = out
+        if kind in GLOBAL_KINDS:
+            if scratch is None:
+                scratch = torch.zeros(blocks * 16384, device=dev)
+            dst = scratch
         for _ in range(2):
-            lib.cvqmb_run(kind, blocks, threads, ITERS[kind] // 10, ctypes.c_void_p(out.data_ptr()),
+            lib.cvqmb_run(kind, blocks, threads, ITERS[kind] // 10, ctypes.c_void_p(dst.data_ptr()),
                           ctypes.c_void_p(stream.cuda_stream))
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        ops = lib.cvqmb_run(kind, blocks, threads, ITERS[kind], ctypes.c_void_p(out.data_ptr()),
+        ops = lib.cvqmb_run(kind, blocks, threads, ITERS[kind], ctypes.c_void_p(dst.data_ptr()),
                             ctypes.c_void_p(stream.cuda_stream))
         e1.record()
         torch.cuda.synchronize()

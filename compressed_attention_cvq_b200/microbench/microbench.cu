@@ -216,11 +216,36 @@ __global__ void rmw_kernel(float* out, int iters, int mode) {
   if (bf[threadIdx.x] + acc.x == 123.456f) out[threadIdx.x] = 1.f;
 }
 
+// Reductions into global memory (L2), each CTA in its own 64 KB window of `buf`
+// (blocks x 16384 floats): mode 0: red.global.add.v4.f32 (16 bytes, one op) at
+// pseudo-random 16-byte slots; 1: red.global.add.f32 at pseudo-random floats; 2: like 0,
+// but every 5th op of a lane goes to one of 4 hot slots (a skewed code distribution).
+__global__ void gred_kernel(float* buf, int iters, int mode) {
+  float* win = buf + static_cast<size_t>(blockIdx.x) * 16384;
+  unsigned x = 2654435761u * (threadIdx.x + 1) + 97u * blockIdx.x;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      x = x * 1664525u + 1013904223u;
+      if (mode == 1) {
+        float* p = win + (x >> 18);                         // 0 .. 16383
+        asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(1.0f) : "memory");
+      } else {
+        unsigned slot = x >> 20;                            // 0 .. 4095
+        if (mode == 2 && (r == 0 || r == 5)) slot &= 3u;    // 2 of 8 ops (25%) on 4 hot slots
+        float* p = win + 4 * slot;
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %1, %1, %1};" ::"l"(p), "f"(1.0f) : "memory");
+      }
+    }
+  }
+}
+
 }  // namespace
 
 // kind: 0 ffma, 1 ffma2, 2 sincos, 3 exp2, 4 lds128 conflict-free, 5 lds128 random,
 //       6 atomic distinct banks, 7 atomic random, 8 atomic same address, 9 shfl,
-//       10..15 rmw_kernel modes 0..5 (mode 5 counts one gather + two reductions as one op)
+//       10..15 rmw_kernel modes 0..5 (mode 5 counts one gather + two reductions as one op),
+//       16..18 gred_kernel modes 0..2 (`out` must hold blocks x 16384 floats)
 // Returns the operation count of the launch (per-thread ops x threads x blocks), or
 // -1 for an unknown kind / launch error.  Operations: FMA lanes (ffma2 counts 2 per
 // instruction), sin+cos pairs, exp2, 16-byte loads, atomics, shuffles.
@@ -241,6 +266,8 @@ MB_API double cvqmb_run(int kind, int blocks, int threads, int iters, float* out
     case 9: shfl_kernel<<<blocks, threads, 0, s>>>(out, iters); per = 32.0 * iters; break;
     case 10: case 11: case 12: case 13: case 14: case 15:
       rmw_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 10); per = 8.0 * iters; break;
+    case 16: case 17: case 18:
+      gred_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 16); per = 8.0 * iters; break;
     default: return -1;
   }
   if (cudaGetLastError() != cudaSuccess) return -1;

@@ -319,7 +319,14 @@ CVQ_API cvq_status cvq_attend_static(const cvq_shape* shape, const void* q, int 
  * cvq_attend_static with 4 query heads per KV head, and every g = 64 decode) wait for
  * those copies with a bounded wait; if a wait gives up, the kernel sets a bit here and
  * runs to completion (its outputs are then invalid) instead of hanging the GPU.
- *   Bits: CVQ_FAULT_COPY_TIMEOUT = a codebook copy did not land within the wait limit.
+ *   Bits: CVQ_FAULT_COPY_TIMEOUT = a codebook copy (or, in a decode kernel, a wait on a
+ *         shared-memory barrier) did not complete within the wait limit;
+ *         CVQ_FAULT_BOUNDS = a device-side range check failed.  Only the debug build of
+ *         the library (compiled with -DCVQ_DEBUG_BOUNDS, libcvq_debug.so) has these checks:
+ *         the code row of every code copy, every codeword and bin index, the exchange index
+ *         between the CTAs of a pair, and the partial-state rows and arrival counter of
+ *         every work unit.  A failed check skips its access (a skipped load reads 0) and
+ *         the kernel runs on; the outputs of that call are then invalid.
  *   flags (host): receives the word.  clear != 0 resets it to 0 afterwards.
  *   Synchronous: waits for the device (cudaMemcpy).  The first call on a device looks up
  *   the word's address (cudaGetSymbolAddress), as the first decode call does; make that
@@ -327,6 +334,7 @@ CVQ_API cvq_status cvq_attend_static(const cvq_shape* shape, const void* q, int 
  *   Errors: CVQ_ERR_NULL (flags NULL), CVQ_ERR_CUDA.
  * ------------------------------------------------------------------------------- */
 #define CVQ_FAULT_COPY_TIMEOUT 1u
+#define CVQ_FAULT_BOUNDS 2u
 CVQ_API cvq_status cvq_fault_status(uint32_t* flags, int clear);
 
 #ifdef __cplusplus

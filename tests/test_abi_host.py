@@ -285,3 +285,25 @@ def test_attend_more_argument_errors():
     assert call(_shape(n_q_heads=24, n_kv_heads=8)) == 4          # 3 query heads per KV head
     assert call(_shape(n_q_heads=30, n_kv_heads=8)) == 2          # not a multiple
     assert call(_shape(batch=70000)) == 2
+
+
+def test_debug_build_exports_every_symbol():
+    """The debug build (device-side range checks) is the same ABI."""
+    path = os.path.join(os.path.dirname(b.LIB_PATH), "libcvq_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libcvq_debug.so not built (python -m compressed_attention_cvq_b200.build --debug-bounds)")
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_fault_bits_match_header_and_decode():
+    src = open(HEADER).read()
+    bits = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (CVQ_FAULT_\w+) (\d+)u", src)}
+    assert bits == {"CVQ_FAULT_COPY_TIMEOUT": b.CVQ_FAULT_COPY_TIMEOUT, "CVQ_FAULT_BOUNDS": b.CVQ_FAULT_BOUNDS}
+    assert b.CVQ_FAULT_COPY_TIMEOUT == 1 and b.CVQ_FAULT_BOUNDS == 2
+    assert b.fault_names(0) == []
+    assert b.fault_names(1) == ["copy_timeout"]
+    assert b.fault_names(2) == ["bounds"]
+    assert b.fault_names(3) == ["copy_timeout", "bounds"]
+    assert b.fault_names(2 | 16) == ["bounds", "0x10"]
