@@ -69,7 +69,8 @@ def sfu_ops(w: workloads.Workload, total_tokens: int):
     return float(total_tokens) * 64, float(total_tokens) * w.n_q_heads
 
 
-def roofline_legs(w: workloads.Workload, total_tokens: int, sm_mhz: float, hbm_gbs: float):
+def roofline_legs(w: workloads.Workload, total_tokens: int, sm_mhz: float, hbm_gbs: float,
+                  code_bits: int = 8):
     """Time (us) of one layer step at each bound: FP32 work at the measured FFMA rate, the
     special-function work at the measured sin/cos and exp2 rates, and the code + codebook
     bytes at the measured HBM copy bandwidth.  The roofline is the slowest of the three."""
@@ -77,15 +78,16 @@ def roofline_legs(w: workloads.Workload, total_tokens: int, sm_mhz: float, hbm_g
     fp32_us = algorithmic_flops(w, total_tokens) / 2 / FFMA_LANES_PER_CLK / clk_hz * 1e6
     sc, ex = sfu_ops(w, total_tokens)
     sfu_us = (sc / SINCOS_PAIRS_PER_CLK + ex / EXP2_PER_CLK) / clk_hz * 1e6
-    hbm_us = code_bytes(w, total_tokens) / (hbm_gbs * 1e9) * 1e6
+    hbm_us = code_bytes(w, total_tokens, code_bits) / (hbm_gbs * 1e9) * 1e6
     return {"fp32_us": fp32_us, "sfu_us": sfu_us, "hbm_us": hbm_us}
 
 
-def code_bytes(w: workloads.Workload, total_tokens: int) -> float:
+def code_bytes(w: workloads.Workload, total_tokens: int, code_bits: int = 8) -> float:
     """Bytes that must come from HBM per layer step: key + value codes of every token of
-    every KV head (one byte per group and round), plus the key and value codebooks of
-    every KV head."""
-    codes = float(total_tokens) * w.n_kv_heads * 2 * w.n_groups * w.R
+    every KV head (one code per group and round, code_bits each: 8 = one byte, 6 = the
+    packed 6-bit layout of 64-entry codebooks), plus the key and value codebooks of every
+    KV head."""
+    codes = float(total_tokens) * w.n_kv_heads * 2 * w.n_groups * w.R * code_bits / 8
     cbs = 2.0 * w.n_kv_heads * w.n_groups * w.R * w.n_codes * w.group_dim * 4
     return codes + cbs
 
@@ -179,11 +181,20 @@ def parity_of(layer0, outputs):
             "tolerance": {"max_abs_err": 2e-3, "lse_rel_err": 1e-4}}
 
 
+def code_bits_of(w: workloads.Workload, args) -> int:
+    """Stored bits per code: --code-bits, else 6 (packed) for 64-entry codebooks and 8 for
+    256-entry ones."""
+    if getattr(args, "code_bits", 0):
+        return args.code_bits
+    return 6 if w.group_dim == 64 else 8
+
+
 def workload_config(w: workloads.Workload, args, total_tokens: int) -> dict:
     """The workload a line measures, identical in the GPU arm and the reference arm."""
     return {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "seq_len": w.t_cap, "R": w.R, "group_dim": w.group_dim,
-            "q_dtype": w.q_dtype, "tokens_per_layer": total_tokens, "append": bool(args.append)}
+            "code_bits": code_bits_of(w, args), "q_dtype": w.q_dtype,
+            "tokens_per_layer": total_tokens, "append": bool(args.append)}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -399,7 +410,16 @@ def run_gpu(args):
             sets[-1].update(new_k=torch.from_numpy(nk).to(dev), new_v=torch.from_numpy(nv).to(dev),
                             pos=(sets[-1]["seq_lens"] - 1).contiguous(), host_new=(nk, nv))
     total_tokens = int(sets[0]["host"]["seq_lens"].sum())
+    cbits = code_bits_of(w, args)
     shape = cvq.shape_of(sets[0]["q"], sets[0]["key_codes"], w.rope_base, w.group_dim)
+    if cbits == 6:
+        # the paper's stored rate: repack every input set's codes to 6 bits (setup, on the
+        # device, outside any timed region)
+        shape.code_bits = 6
+        for st_ in sets:
+            st_["key_codes"] = cvq.pack_codes6(shape, st_["key_codes"])
+            st_["val_codes"] = cvq.pack_codes6(shape, st_["val_codes"])
+        torch.cuda.synchronize()
     if args.splits:
         S = args.splits
     elif args.form == "naive":
@@ -507,8 +527,10 @@ def run_gpu(args):
         hq = torch.from_numpy(h["q"])
     host_in = dict(q=hq.pin_memory(), key_cb=torch.from_numpy(h["key_cb"]).pin_memory(),
                    val_cb=torch.from_numpy(h["val_cb"]).pin_memory(),
-                   key_codes=torch.from_numpy(h["key_codes"]).pin_memory(),
-                   val_codes=torch.from_numpy(h["val_codes"]).pin_memory(),
+                   key_codes=(sets[0]["key_codes"].cpu() if cbits == 6
+                              else torch.from_numpy(h["key_codes"])).pin_memory(),
+                   val_codes=(sets[0]["val_codes"].cpu() if cbits == 6
+                              else torch.from_numpy(h["val_codes"])).pin_memory(),
                    seq_lens=torch.from_numpy(h["seq_lens"]).pin_memory())
     if args.append:
         host_in.update(new_k=torch.from_numpy(sets[0]["host_new"][0]).pin_memory(),
@@ -566,7 +588,7 @@ def run_gpu(args):
         else:
             o, l = cvq.attend(d_in["q"], d_in["key_cb"], d_in["val_cb"], d_in["key_codes"],
                               d_in["val_codes"], d_in["seq_lens"], w.rope_base, n_splits=S,
-                              form=args.form)
+                              form=args.form, code_bits=shape.code_bits)
         host_out.copy_(o, non_blocking=True)
         host_lse.copy_(l, non_blocking=True)
         freed[slot].record(stream)
@@ -598,12 +620,12 @@ def run_gpu(args):
         dec_mean_ms = statistics.mean(dec_ms)
         sm_max = pk.get("sm_max_mhz", 1965.0) or 1965.0
         fp32_peak_tflops = SM_COUNT_B200 * FFMA_LANES_PER_CLK * 2 * sm_max * 1e6 / 1e12
-        legs = roofline_legs(w, total_tokens, sm_max, pk["hbm_gbs"])
+        legs = roofline_legs(w, total_tokens, sm_max, pk["hbm_gbs"], cbits)
         bound_leg = max(legs, key=legs.get)
         bound = {"fp32_us": "alu", "sfu_us": "sfu", "hbm_us": "hbm"}[bound_leg]
         flops = algorithmic_flops(w, total_tokens)
         achieved_tflops = flops / (dec_mean_ms * 1e-3) / 1e12
-        bytes_ = code_bytes(w, total_tokens)
+        bytes_ = code_bytes(w, total_tokens, cbits)
         value = whole_job_rate(world, total_tokens, ms_per_step)
         result = {
             "metric": METRIC,
@@ -621,7 +643,7 @@ def run_gpu(args):
             "config": workload_config(w, args, total_tokens),
             "run": {"form": args.form, "n_splits": S,
                     "l2": f"{N_INPUT_SETS} rotating layer input sets of "
-                          f"{code_bytes(w, total_tokens) / 1e6:.0f} MB (> 126 MB L2 in total)",
+                          f"{code_bytes(w, total_tokens, cbits) / 1e6:.0f} MB (> 126 MB L2 in total)",
                     "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "decode_ms": dec_mean_ms,
             "decode_ms_median": statistics.median(dec_ms),
@@ -709,6 +731,9 @@ def main(argv=None):
                          "combine as two launches; table: the pages' per-query-head table "
                          "form; naive: decode the cache to fp16 then attend (comparison path)")
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--code-bits", type=int, choices=[6, 8], default=0,
+                    help="stored bits per code: 6 = packed (64-entry codebooks only); "
+                         "default 6 for 64-entry codebooks, 8 otherwise")
     ap.add_argument("--append", action="store_true",
                     help="each step first encodes the step's new key/value into the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -77,15 +77,30 @@ def group_dim_of(key_cb):
     return 2 * int(key_cb.shape[-2])
 
 
-def shape_of(q, key_codes, rope_base=500000.0, group_dim=8):
-    """cvq_shape from q [B, Hq, 128] and key_codes: [B, Hkv, T_cap, R, 16] (group_dim 8)
-    or planar [B, Hkv, 2, R, T_cap] (group_dim 64)."""
+def shape_of(q, key_codes, rope_base=500000.0, group_dim=8, code_bits=0):
+    """cvq_shape from q [B, Hq, 128] and key_codes: [B, Hkv, T_cap, R, 16] (group_dim 8),
+    planar [B, Hkv, 2, R, T_cap] (group_dim 64) or, with code_bits 6, packed planar
+    [B, Hkv, 2, R, 3 T_cap / 4]."""
     B, Hq, D = q.shape
     if group_dim == 64:
         _, Hkv, _, R, T = key_codes.shape
+        if code_bits == 6:
+            T = T * 4 // 3
     else:
         _, Hkv, T, R, _ = key_codes.shape
-    return make_shape(B, Hq, Hkv, R, T, rope_base, D, group_dim)
+    return make_shape(B, Hq, Hkv, R, T, rope_base, D, group_dim, code_bits)
+
+
+def pack_codes6(shape, codes, out=None, stream=None):
+    """cvq_pack_codes6: planar one-byte codes [B, Hkv, 2, R, T_cap] -> packed 6-bit
+    [B, Hkv, 2, R, 3 T_cap / 4] uint8 (shape: group_dim 64, code_bits 6)."""
+    _require(codes, "codes", torch.uint8)
+    if out is None:
+        out = torch.empty((*codes.shape[:-1], codes.shape[-1] // 4 * 3), dtype=torch.uint8,
+                          device=codes.device)
+    st = _b.lib.cvq_pack_codes6(ctypes.byref(shape), _ptr(codes), _ptr(out), _stream(stream))
+    _b.check(st, "cvq_pack_codes6")
+    return out
 
 
 def split_tokens(shape, n_splits):
@@ -261,15 +276,16 @@ def naive_decode(shape, q, k, v, seq_lens, n_splits, partials=None, stream=None)
 
 
 def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, rope_base=500000.0, n_splits=None,
-           form="gqa", stream=None):
+           form="gqa", stream=None, code_bits=0):
     """One decode step: (out [B, Hq, 128], lse [B, Hq]) in fp32.
 
     form="gqa":   cvq_attend (decode with the merge fused in: one launch)
     form="gqa_split": cvq_decode_attn_gqa + cvq_combine
     form="table": cvq_qtable + cvq_decode_attn + cvq_combine
     form="naive": cvq_naive_dequant + cvq_naive_decode + cvq_combine (the comparison path)
+    code_bits=6: the codes are packed 6-bit rows (64-scalar groups; see pack_codes6).
     """
-    shape = shape_of(q, key_codes, rope_base, group_dim_of(key_cb))
+    shape = shape_of(q, key_codes, rope_base, group_dim_of(key_cb), code_bits)
     if n_splits is None:
         n_splits = suggest_splits(shape)
     if form == "table":

@@ -32,7 +32,7 @@ class cvq_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("R", ctypes.c_int32), ("t_cap", ctypes.c_int32), ("rope_base", ctypes.c_float),
-                ("group_dim", ctypes.c_int32)]
+                ("group_dim", ctypes.c_int32), ("code_bits", ctypes.c_int32)]
 
 
 def _load():
@@ -61,6 +61,7 @@ def _load():
         "cvq_attend_workspace_bytes": (SZ, [S, I]),
         "cvq_attend": (I, [S, P, I, P, I64, P, P, P, P, I64, I, P, P, P, P]),
         "cvq_fault_status": (I, [ctypes.POINTER(ctypes.c_uint32), I]),
+        "cvq_pack_codes6": (I, [S, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -88,7 +89,7 @@ EXPORTED = ["cvq_status_str", "cvq_abi_version", "cvq_ptable_bytes", "cvq_partia
             "cvq_decode_attn_gqa", "cvq_combine", "cvq_attend_static",
             "cvq_naive_cache_bytes", "cvq_naive_dequant", "cvq_naive_decode",
             "cvq_encode_append", "cvq_attend_workspace_bytes", "cvq_attend",
-            "cvq_fault_status"]
+            "cvq_fault_status", "cvq_pack_codes6"]
 CVQ_FAULT_COPY_TIMEOUT = 1
 CVQ_FAULT_BOUNDS = 2
 FAULT_NAMES = {CVQ_FAULT_COPY_TIMEOUT: "copy_timeout", CVQ_FAULT_BOUNDS: "bounds"}
@@ -111,5 +112,6 @@ def check(st: int, what: str):
 
 
 def make_shape(batch, n_q_heads, n_kv_heads, R, t_cap, rope_base=500000.0, head_dim=128,
-               group_dim=8):
-    return cvq_shape(batch, n_q_heads, n_kv_heads, head_dim, R, t_cap, rope_base, group_dim)
+               group_dim=8, code_bits=0):
+    return cvq_shape(batch, n_q_heads, n_kv_heads, head_dim, R, t_cap, rope_base, group_dim,
+                     code_bits)

@@ -30,11 +30,17 @@ cvq_status check_shape(const cvq_shape* s) {
   if (s->head_dim != kHeadDim) return CVQ_ERR_UNSUPPORTED;
   if (s->group_dim != 0 && s->group_dim != 8 && s->group_dim != kWideGroupDim)
     return CVQ_ERR_UNSUPPORTED;
+  if (s->code_bits != 0 && s->code_bits != 8 && s->code_bits != 6) return CVQ_ERR_UNSUPPORTED;
   if (is_wide(s)) {
     if (s->R < 1 || s->R > kWideMaxR) return CVQ_ERR_UNSUPPORTED;
     if (s->t_cap % 16 != 0) return CVQ_ERR_SHAPE;      // planar code rows in 16-byte chunks
+    // packed rows: 64 codes = 48 bytes, so every row and every 64-token chunk of it
+    // starts on a 16-byte boundary
+    if (s->code_bits == 6 && s->t_cap % 64 != 0) return CVQ_ERR_SHAPE;
   } else if (s->R != 1 && s->R != 2) {
     return CVQ_ERR_UNSUPPORTED;
+  } else if (s->code_bits == 6) {
+    return CVQ_ERR_UNSUPPORTED;                        // 6-bit codes: 64-entry codebooks only
   }
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->t_cap < 0) return CVQ_ERR_SHAPE;
   if (s->n_q_heads % s->n_kv_heads != 0) return CVQ_ERR_SHAPE;
@@ -95,6 +101,7 @@ void fill_common(DecodeArgs& a, const cvq_shape* s, const uint8_t* key_codes, co
   a.n_q_heads = s->n_q_heads;
   a.n_kv_heads = s->n_kv_heads;
   a.t_cap = s->t_cap;
+  a.code_bits = s->code_bits == 6 ? 6 : 8;
   a.n_splits = n_splits;
   a.split_tokens = split_tokens_host(s->t_cap, n_splits);
   a.part_o = part_o;
@@ -387,6 +394,18 @@ cvq_status cvq_naive_decode(const cvq_shape* s, const void* q, int q_dtype, cons
   return from_cuda(launch_naive_decode(*s, q, q_dtype, k, v, seq_lens, n_splits,
                                        split_tokens_host(s->t_cap, n_splits), part_o, part_m,
                                        part_l, static_cast<cudaStream_t>(stream)));
+}
+
+cvq_status cvq_pack_codes6(const cvq_shape* s, const uint8_t* codes_in, uint8_t* packed_out,
+                           void* stream) {
+  CVQ_TRY(check_shape(s));
+  if (!is_wide(s) || s->code_bits != 6) return CVQ_ERR_UNSUPPORTED;
+  CVQ_TRY(check_ptr(codes_in));
+  CVQ_TRY(check_ptr(packed_out));
+  if (s->t_cap == 0) return CVQ_OK;
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_kv_heads * kWideGroups * s->R;
+  return from_cuda(launch_pack_codes6(codes_in, packed_out, rows, s->t_cap,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 cvq_status cvq_encode_append(const cvq_shape* s, const float* keys, const float* values,

@@ -78,6 +78,17 @@ __device__ __forceinline__ float load_q(const void* q, int q_dtype, size_t idx) 
   return static_cast<const float*>(q)[idx];
 }
 
+// Code t of a packed row (6 bits per code, 4 codes in 3 bytes, little-endian: code
+// 4i + j in bits 6j .. 6j+5 of the 24-bit word in bytes 3i .. 3i+2).  A code lies in one
+// byte (j = 0, 3) or two bytes of its own 3-byte group (j = 1, 2); nothing past the
+// group is read.
+__device__ __forceinline__ int packed6_code(const uint8_t* row, int t) {
+  const int bit = 6 * t, by = bit >> 3, sh = bit & 7;
+  uint32_t w = row[by];
+  if (sh > 2) w |= static_cast<uint32_t>(row[by + 1]) << 8;
+  return static_cast<int>((w >> sh) & 63u);
+}
+
 __device__ __forceinline__ int code_byte(const uint4& v, int G) {
   const uint32_t w = (G < 4) ? v.x : (G < 8) ? v.y : (G < 12) ? v.z : v.w;
   return static_cast<int>((w >> (8 * (G & 3))) & 0xffu);
@@ -103,6 +114,7 @@ struct DecodeArgs {
   const float* val_cb;
   long long val_cb_stride;
   int batch, n_q_heads, n_kv_heads, t_cap, n_splits, split_tokens;
+  int code_bits;                 // 8: one byte per code; 6: packed (64-scalar groups only)
   float* part_o;
   float* part_m;
   float* part_l;
@@ -365,6 +377,9 @@ cvq_status attend_into(const cvq_shape* s, const void* q, int q_dtype, const flo
                        const uint8_t* val_codes, const int32_t* seq_lens, const float* val_cb,
                        int64_t val_cb_head_stride, int n_splits, float* partials, int* counters,
                        float* out, float* lse, void* stream, size_t clear_counters);
+// 6-bit packing of `rows` planar code rows of t_cap codes each (pack.cu)
+cudaError_t launch_pack_codes6(const uint8_t* codes_in, uint8_t* packed_out, size_t rows, int t_cap,
+                               cudaStream_t stream);
 cudaError_t launch_combine(const cvq_shape& s, int n_splits, const float* part_o,
                            const float* part_m, const float* part_l, float* out, float* lse,
                            cudaStream_t stream);

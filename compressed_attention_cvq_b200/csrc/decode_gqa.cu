@@ -29,9 +29,9 @@
 //     touch 32 different banks and never the same address.
 //
 // Tokens: kSlots = 4 per warp per step; slot sigma handles t_begin + sigma + kSlots*j.
-// The phase of a lane's 4 pairs is re-seeded from the exact fixed-point turn at the start
-// of every tile and advances by e^{i theta_j kSlots} per step within it (at most
-// kSteps - 1 products, rounding error ~1e-7 each).  Code bytes of the
+// The phase of a lane's 4 pairs is re-seeded from the exact fixed-point turn every 8
+// steps (every tile at R = 1, every second tile at R = 2) and advances by
+// e^{i theta_j kSlots} per step in between (at most 7 products, rounding error ~1e-7 each).  Code bytes of the
 // next tile are copied to shared memory with cp.async while the current tile computes.
 #include <cooperative_groups.h>
 
@@ -65,6 +65,12 @@ struct Cfg {
                                   sizeof(float) * (kBins + kXchg + kWarps * kHeads + 4 * kHeads) +
                                   kCodeBytes + 16;   // + the TMA mbarrier
   static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
+  // the RoPE phase is re-seeded exactly every kReseedSteps steps (every tile at R = 1, every
+  // second tile at R = 2), so at most kReseedSteps - 1 recurrence products separate a phase
+  // from its exact seed
+  static constexpr int kReseedSteps = 8;
+  static constexpr int kReseedTiles = kReseedSteps / kSteps;
+  static_assert(kReseedTiles * kSteps == kReseedSteps, "whole tiles between seeds");
 };
 
 __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
@@ -200,8 +206,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
                              load_q(a.q, a.q_dtype, qb + 2 * pp + 1) * qscale);
     }
   }
-  // phase of the lane's pairs: re-seeded from the exact turn at the first token of every
-  // tile, advanced by e^{i theta kSlots} per step within the tile (<= kSteps - 1 products)
+  // phase of the lane's pairs: re-seeded from the exact turn every kReseedSteps steps,
+  // advanced by e^{i theta kSlots} per step in between
   float2 ph[4], adv[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) adv[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], C::kSlots);
@@ -299,8 +305,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     float* xb = xchg + buf * (kTile * kHeads);
     float* pxb = peer_xchg + buf * (kTile * kHeads);
 
+    if (tile % C::kReseedTiles == 0) {   // exact seed at least every kReseedSteps steps
 #pragma unroll
-    for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
+      for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
+    }
     float s_part[C::kSteps];
     constexpr int kGS = C::kSteps >= 4 ? 4 : C::kSteps;   // steps per pass group
 #pragma unroll

@@ -147,15 +147,22 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
 
   // planar codes: row (b, h, G, r) of t_cap bytes
   const size_t code_row0 = ((static_cast<size_t>(b) * a.n_kv_heads + h) * kWideGroups + G) * R + r0;
+  // a code row holds t_cap bytes, or 3 t_cap / 4 packed (t_cap and every tile start a
+  // multiple of 64, so a tile's packed bytes start on a 16-byte boundary); the tile's
+  // 16-byte chunks that hold tokens before t_end are copied, never past the row's end
+  const bool packed6 = a.code_bits == 6;
+  const size_t row_bytes = packed6 ? static_cast<size_t>(a.t_cap) / 4 * 3 : static_cast<size_t>(a.t_cap);
+  constexpr int kChunksPerRow = kWTile / 16;           // unpacked; packed uses 3/4 of them
   auto stage_codes = [&](int t_tile, int buf) {
-    const int n = 2 * rc * (kWTile / 16);
+    const int n = 2 * rc * kChunksPerRow;
+    const size_t tile_byte = packed6 ? static_cast<size_t>(t_tile) / 4 * 3 : static_cast<size_t>(t_tile);
+    const int need = packed6 ? ((t_end - t_tile) * 3 + 3) / 4 : (t_end - t_tile);   // bytes with tokens < t_end
     for (int i = tid; i < n; i += kWThreads) {
-      const int kind = i / (rc * (kWTile / 16));
-      const int r = (i / (kWTile / 16)) % rc;
-      const int q16 = i % (kWTile / 16);
-      const int t = t_tile + 16 * q16;
-      if (t < t_end && in_bounds(a.fault, t + 15, a.t_cap)) {
-        const uint8_t* src = (kind ? a.val_codes : a.key_codes) + (code_row0 + r) * a.t_cap + t;
+      const int kind = i / (rc * kChunksPerRow);
+      const int r = (i / kChunksPerRow) % rc;
+      const int q16 = i % kChunksPerRow;
+      if (16 * q16 < need && in_bounds(a.fault, tile_byte + 16 * q16 + 15, row_bytes)) {
+        const uint8_t* src = (kind ? a.val_codes : a.key_codes) + (code_row0 + r) * row_bytes + tile_byte + 16 * q16;
         cp_async16(code_s + ((buf * 2 + kind) * kRC + r) * kWTile + 16 * q16, src);
       }
     }
@@ -222,9 +229,14 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
       const int kind = tid >> 8, t = tid & 255;
       const uint8_t* src = code_s + (buf * 2 + kind) * kRC * kWTile + t;
       uint32_t wv[4] = {0u, 0u, 0u, 0u};
+      const uint8_t* srow = code_s + (buf * 2 + kind) * kRC * kWTile;     // packed rows
 #pragma unroll
       for (int r = 0; r < kRC; ++r)
-        if (r < rc) wv[r >> 2] |= static_cast<uint32_t>(src[r * kWTile]) << (8 * (r & 3));
+        if (r < rc) {
+          const uint32_t c = packed6 ? static_cast<uint32_t>(packed6_code(srow + r * kWTile, t))
+                                     : static_cast<uint32_t>(src[r * kWTile]);
+          wv[r >> 2] |= c << (8 * (r & 3));
+        }
       *reinterpret_cast<uint4*>(tcode + (kind * kWTile + t) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     __syncthreads();

@@ -96,16 +96,19 @@ __global__ void __launch_bounds__(32 * kEncWarps) encode_kernel(
 }
 
 // The paper's layout: 2 groups of 64 scalars, 64 codewords per (group, round), planar codes
-// [B, Hkv, 2, R, t_cap].  One warp per (sequence x KV head, key | value, group); lane l scores
-// codewords l and l + 32.  The residual (64 floats) sits in shared memory and every lane
-// reads it in dim order 0..63, so each distance is summed in one fixed order.
+// [B, Hkv, 2, R, t_cap], one byte per code, or (packed6) 4 codes in 3 bytes per row, where
+// only the 6 bits of the written code change (a read-modify-write of its one or two bytes;
+// no other thread writes the row in the same call).  One warp per (sequence x KV head,
+// key | value, group); lane l scores codewords l and l + 32.  The residual (64 floats) sits
+// in shared memory and every lane reads it in dim order 0..63, so each distance is summed
+// in one fixed order.
 constexpr int kWideEncWarps = 8;
 
 __global__ void __launch_bounds__(32 * kWideEncWarps) encode_wide_kernel(
     const float* __restrict__ keys, const float* __restrict__ values,
     const float* __restrict__ key_cb, long long key_stride, const float* __restrict__ val_cb,
     long long val_stride, const int32_t* __restrict__ positions, uint8_t* __restrict__ key_codes,
-    uint8_t* __restrict__ val_codes, int R, int n_kv_heads, int t_cap, int n_units) {
+    uint8_t* __restrict__ val_codes, int R, int n_kv_heads, int t_cap, int n_units, bool packed6) {
   __shared__ __align__(16) float res_s[kWideEncWarps][kWideVDims];
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int unit = blockIdx.x * kWideEncWarps + wl;             // (bh, is_val, G)
@@ -117,8 +120,8 @@ __global__ void __launch_bounds__(32 * kWideEncWarps) encode_wide_kernel(
   const float* src = (is_val ? values : keys) + static_cast<size_t>(bh) * kHeadDim + kWideVDims * G;
   const float* cb = (is_val ? val_cb + h * val_stride : key_cb + h * key_stride) +
                     static_cast<size_t>(G) * R * kWideCodes * kWideVDims;
-  uint8_t* out = (is_val ? val_codes : key_codes) +
-                 ((static_cast<size_t>(bh) * kWideGroups + G) * R) * t_cap + p;
+  const size_t row_bytes = packed6 ? static_cast<size_t>(t_cap) / 4 * 3 : static_cast<size_t>(t_cap);
+  uint8_t* rows = (is_val ? val_codes : key_codes) + ((static_cast<size_t>(bh) * kWideGroups + G) * R) * row_bytes;
   float* res = res_s[wl];
   res[lane] = src[lane];
   res[lane + 32] = src[lane + 32];
@@ -151,7 +154,20 @@ __global__ void __launch_bounds__(32 * kWideEncWarps) encode_wide_kernel(
       const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
       if (od < bd || (od == bd && oc < bc)) { bd = od; bc = oc; }
     }
-    if (lane == 0) out[static_cast<size_t>(r) * t_cap] = static_cast<uint8_t>(bc);
+    if (lane == 0) {
+      uint8_t* row = rows + static_cast<size_t>(r) * row_bytes;
+      if (packed6) {
+        // code p: bits 6p .. 6p+5 of the row, in byte 6p / 8 and, past bit 2 of it, the next
+        const int bit = 6 * p, by = bit >> 3, sh = bit & 7;
+        uint32_t w = row[by];
+        if (sh > 2) w |= static_cast<uint32_t>(row[by + 1]) << 8;
+        w = (w & ~(63u << sh)) | (static_cast<uint32_t>(bc) << sh);
+        row[by] = static_cast<uint8_t>(w);
+        if (sh > 2) row[by + 1] = static_cast<uint8_t>(w >> 8);
+      } else {
+        row[p] = static_cast<uint8_t>(bc);
+      }
+    }
     const float* chosen = cb + (static_cast<size_t>(r) * kWideCodes + bc) * kWideVDims;
     const float n0 = __fsub_rn(res[lane], __ldg(chosen + lane));
     const float n1 = __fsub_rn(res[lane + 32], __ldg(chosen + lane + 32));
@@ -173,7 +189,7 @@ cudaError_t launch_encode_append(const cvq_shape& s, const float* keys, const fl
     const unsigned blocks = static_cast<unsigned>((n_units + kWideEncWarps - 1) / kWideEncWarps);
     encode_wide_kernel<<<blocks, 32 * kWideEncWarps, 0, stream>>>(
         keys, values, key_cb, key_stride, val_cb, val_stride, positions, key_codes, val_codes,
-        s.R, s.n_kv_heads, s.t_cap, n_units);
+        s.R, s.n_kv_heads, s.t_cap, n_units, s.code_bits == 6);
     return cudaGetLastError();
   }
   // units = B * Hkv * 2 * 16, a multiple of kEncWarps

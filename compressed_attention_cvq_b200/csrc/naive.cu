@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kDqThreads) naive_dequant_kernel(
 }
 
 // The same for the paper's layout (2 groups of 64 scalars, 64 codewords, planar codes
-// [B, Hkv, 2, R, t_cap]): block (32 tokens, 8 chunks) per (token block, KV head x group,
+// [B, Hkv, 2, R, t_cap], or packed 6-bit rows of 3 t_cap / 4 bytes when packed6): block
+// (32 tokens, 8 chunks) per (token block, KV head x group,
 // sequence); thread (token, chunk) sums the R codewords' 8-float chunk of its group for
 // the key (pairs 32 G + 4 chunk .. + 3, rotated) and the value (dims 64 G + 8 chunk ..).
 __global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
     long long val_stride, const uint8_t* __restrict__ key_codes,
     const uint8_t* __restrict__ val_codes, const int32_t* __restrict__ seq_lens, int R,
     int n_kv_heads, int t_cap, PhaseTurns phase, __half* __restrict__ k_out,
-    __half* __restrict__ v_out) {
+    __half* __restrict__ v_out, bool packed6) {
   const int t = blockIdx.x * 32 + threadIdx.x;
   const int chunk = threadIdx.y;
   const int G = blockIdx.y & 1, h = blockIdx.y >> 1, b = blockIdx.z;
@@ -78,16 +79,19 @@ __global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
   L = L < 0 ? 0 : (L > t_cap ? t_cap : L);
   if (t >= L) return;
   const size_t bh = static_cast<size_t>(b) * n_kv_heads + h;
-  const uint8_t* kc = key_codes + (bh * kWideGroups + G) * R * static_cast<size_t>(t_cap) + t;
-  const uint8_t* vc = val_codes + (bh * kWideGroups + G) * R * static_cast<size_t>(t_cap) + t;
+  const size_t row_bytes = packed6 ? static_cast<size_t>(t_cap) / 4 * 3 : static_cast<size_t>(t_cap);
+  const uint8_t* kc = key_codes + (bh * kWideGroups + G) * R * row_bytes;
+  const uint8_t* vc = val_codes + (bh * kWideGroups + G) * R * row_bytes;
   const float* kcb = key_cb + h * key_stride + static_cast<size_t>(G) * R * kWideCodes * kWideVDims + 8 * chunk;
   const float* vcb = val_cb + h * val_stride + static_cast<size_t>(G) * R * kWideCodes * kWideVDims + 8 * chunk;
   float k[8], v[8];
 #pragma unroll
   for (int d = 0; d < 8; ++d) k[d] = v[d] = 0.f;
   for (int r = 0; r < R; ++r) {
-    const int ck = kc[static_cast<size_t>(r) * t_cap] & (kWideCodes - 1);
-    const int cv = vc[static_cast<size_t>(r) * t_cap] & (kWideCodes - 1);
+    const uint8_t* krow = kc + static_cast<size_t>(r) * row_bytes;
+    const uint8_t* vrow = vc + static_cast<size_t>(r) * row_bytes;
+    const int ck = packed6 ? packed6_code(krow, t) : (krow[t] & (kWideCodes - 1));
+    const int cv = packed6 ? packed6_code(vrow, t) : (vrow[t] & (kWideCodes - 1));
     const float4* kw = reinterpret_cast<const float4*>(kcb + (static_cast<size_t>(r) * kWideCodes + ck) * kWideVDims);
     const float4* vw = reinterpret_cast<const float4*>(vcb + (static_cast<size_t>(r) * kWideCodes + cv) * kWideVDims);
     const float4 a0 = __ldg(kw), a1 = __ldg(kw + 1), b0 = __ldg(vw), b1 = __ldg(vw + 1);
@@ -121,7 +125,8 @@ cudaError_t launch_naive_dequant(const cvq_shape& s, const float* key_cb, long l
     dim3 grid((s.t_cap + 31) / 32, s.n_kv_heads * kWideGroups, s.batch);
     naive_dequant_wide_kernel<<<grid, dim3(32, 8), 0, stream>>>(
         key_cb, key_stride, val_cb, val_stride, key_codes, val_codes, seq_lens, s.R,
-        s.n_kv_heads, s.t_cap, phase, static_cast<__half*>(k_out), static_cast<__half*>(v_out));
+        s.n_kv_heads, s.t_cap, phase, static_cast<__half*>(k_out), static_cast<__half*>(v_out),
+        s.code_bits == 6);
     return cudaGetLastError();
   }
   dim3 grid((s.t_cap + kDqThreads / 16 - 1) / (kDqThreads / 16), s.n_kv_heads, s.batch);

@@ -21,7 +21,10 @@
  *          "Limitations"): key 2 groups of 32 pairs, value 2 groups of 64 dims, 64
  *          codewords per (group, round), R = 1..22 (11 -> 1.03 bits, 21 -> 1.97 bits
  *          per scalar; each 6-bit code is stored in one uint8);
- *          codes planar [B, Hkv, 2, R, t_cap], t_cap a multiple of 16.
+ *          codes planar [B, Hkv, 2, R, t_cap], t_cap a multiple of 16, one byte per
+ *          code; or, with code_bits = 6, packed 4 codes in 3 bytes along each row
+ *          (planar [B, Hkv, 2, R, 3 t_cap / 4] bytes, t_cap a multiple of 64), which
+ *          stores exactly R x 6 / 64 bits per scalar.
  *   score_t = sum_j Re(e^{i theta_j t} conj(q_j) sum_r c_{t,r,j}) / sqrt(128), t = 0..L-1
  *   out = sum_t softmax(score)_t v_t,   lse = ln sum_t exp(score_t).
  * Query head hq reads KV head hq / (n_q_heads / n_kv_heads).
@@ -63,7 +66,7 @@ extern "C" {
 #define CVQ_API
 #endif
 
-#define CVQ_ABI_VERSION 2
+#define CVQ_ABI_VERSION 3
 #define CVQ_HEAD_DIM 128
 #define CVQ_GROUPS 16
 #define CVQ_CODES 256
@@ -90,6 +93,9 @@ typedef struct {
   int32_t t_cap;      /* token capacity of the code buffers per sequence, >= 0 */
   float rope_base;    /* RoPE base, > 1 (500000 for LLaMA-3.1)                */
   int32_t group_dim;  /* scalars per quantization group: 0 or 8 (default), 64 */
+  int32_t code_bits;  /* storage of a code: 0 or 8 = one byte per code (default);
+                         6 = packed, 4 codes in 3 bytes (group_dim 64 only, t_cap a
+                         multiple of 64; see cvq_pack_codes6)                   */
 } cvq_shape;
 
 /* Human-readable name of a status code (static storage). */
@@ -174,7 +180,9 @@ CVQ_API cvq_status cvq_decode_attn(const cvq_shape* shape, const float* ptable, 
  *     val_cb     [Hkv][2, R, 64, 64] fp32 (value dim 64 G + d), same stride rule
  *     key_codes, val_codes  planar [B, Hkv, 2, R, t_cap] uint8 (the low 6 bits of
  *                each byte are the code; the top 2 bits are ignored), t_cap a multiple
- *                of 16 (else CVQ_ERR_SHAPE)
+ *                of 16 (else CVQ_ERR_SHAPE); with code_bits = 6 packed planar
+ *                [B, Hkv, 2, R, 3 t_cap / 4] bytes (layout at cvq_pack_codes6), t_cap a
+ *                multiple of 64 (else CVQ_ERR_SHAPE)
  * ------------------------------------------------------------------------------- */
 CVQ_API cvq_status cvq_decode_attn_gqa(const cvq_shape* shape, const void* q, int q_dtype,
                                const float* key_cb, int64_t key_cb_head_stride,
@@ -269,8 +277,11 @@ CVQ_API cvq_status cvq_naive_decode(const cvq_shape* shape, const void* q, int q
  *                 outside [0, t_cap) writes nothing for that sequence
  *   key_codes, val_codes  [B, Hkv, t_cap, R, 16] uint8, written at [b, h, positions[b]]
  *                 (group_dim = 64: planar [B, Hkv, 2, R, t_cap], written at
- *                 [b, h, :, :, positions[b]]) and nowhere else (the caller owns them; seq_lens is the caller's to
- *                 advance)
+ *                 [b, h, :, :, positions[b]]; with code_bits = 6 the packed planar rows,
+ *                 where only the 6 bits of code positions[b] change in each row) and
+ *                 nowhere else (the caller owns them; seq_lens is the caller's to
+ *                 advance).  Calls that write the same rows must be ordered on one
+ *                 stream (a packed code shares its bytes with its neighbours).
  *   Errors: CVQ_ERR_NULL / CVQ_ERR_ALIGN / CVQ_ERR_SHAPE / CVQ_ERR_UNSUPPORTED before any
  *   launch; CVQ_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
  * ------------------------------------------------------------------------------- */
@@ -279,6 +290,25 @@ CVQ_API cvq_status cvq_encode_append(const cvq_shape* shape, const float* keys, 
                                      const float* val_cb, int64_t val_cb_head_stride,
                                      const int32_t* positions, uint8_t* key_codes,
                                      uint8_t* val_codes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * cvq_pack_codes6 -- repack the paper's 6-bit codes from one byte per code to 4 codes in
+ * 3 bytes (CommVQ summary page, "Key results": 64-entry codebooks, so R = 11 rounds
+ * over 64-scalar groups store 11 x 6 / 64 = 1.03 bits per scalar).  The pages fix no bit
+ * layout; this one is little-endian along each row of the planar layout: codes
+ * t = 4i .. 4i+3 of a (sequence, KV head, group, round) row form the 24-bit
+ * little-endian word in bytes 3i .. 3i+2, code 4i + j in bits 6j .. 6j+5.
+ *   shape      group_dim 64, code_bits 6 (the layout being produced), t_cap a multiple
+ *              of 64
+ *   codes_in   planar [B, Hkv, 2, R, t_cap] uint8, one code per byte (low 6 bits used),
+ *              16-byte aligned
+ *   packed_out planar [B, Hkv, 2, R, 3 t_cap / 4] uint8, 16-byte aligned; every byte
+ *              is written (every token up to t_cap, whatever the sequence lengths)
+ *   Errors: CVQ_ERR_NULL / CVQ_ERR_ALIGN / CVQ_ERR_SHAPE / CVQ_ERR_UNSUPPORTED before any
+ *   launch; CVQ_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------------- */
+CVQ_API cvq_status cvq_pack_codes6(const cvq_shape* shape, const uint8_t* codes_in,
+                                   uint8_t* packed_out, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * cvq_attend_static -- cvq_attend (decode with the fused split merge, one launch) with

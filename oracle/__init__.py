@@ -3,4 +3,4 @@
 Only the tests, the smoke check and the benchmark's CPU-baseline leg may import this
 package.  It shares no code with the CUDA library and the library never imports it.
 """
-from . import brute, cvq_oracle, encode  # noqa: F401
+from . import brute, cvq_oracle, encode, pack  # noqa: F401

@@ -182,8 +182,14 @@ def attend(q, key_cb, val_cb, key_codes, val_codes, seq_lens, base, heads=None,
     """Full decode step.  Returns out [B, Hq, 128] and lse [B, Hq] (float64).
 
     `heads`, if given, is an iterable of (b, hq) to compute; other entries are NaN.
-    `codes_layout` "planar" takes codes as [B, Hkv, NG, R, T_cap].
+    `codes_layout` "planar" takes codes as [B, Hkv, NG, R, T_cap]; "planar6" takes them
+    packed 6 bits per code along the token axis (oracle/pack.py), [B, Hkv, NG, R, 3 T_cap/4].
     """
+    if codes_layout == "planar6":
+        from .pack import unpack_codes6
+        n = key_codes.shape[-1] * 4 // 3
+        key_codes, val_codes = unpack_codes6(key_codes, n), unpack_codes6(val_codes, n)
+        codes_layout = "planar"
     if codes_layout == "planar":
         key_codes, val_codes = token_major(key_codes), token_major(val_codes)
     q = np.asarray(q, dtype=np.float64)

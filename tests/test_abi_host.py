@@ -307,3 +307,33 @@ def test_fault_bits_match_header_and_decode():
     assert b.fault_names(2) == ["bounds"]
     assert b.fault_names(3) == ["copy_timeout", "bounds"]
     assert b.fault_names(2 | 16) == ["bounds", "0x10"]
+
+
+def test_packed_code_layout_validation():
+    """code_bits: 0 / 8 one byte per code, 6 packed (64-scalar groups only, t_cap a multiple
+    of 64); every error is returned before any launch (fake pointers are never touched)."""
+    s = _shape(group_dim=64, R=11, t_cap=1024, n_q_heads=8, n_kv_heads=2)
+    s.code_bits = 6
+    # sizes do not depend on the code storage
+    s8 = _shape(group_dim=64, R=11, t_cap=1024, n_q_heads=8, n_kv_heads=2)
+    assert b.lib.cvq_partials_bytes(ctypes.byref(s), 4) == b.lib.cvq_partials_bytes(ctypes.byref(s8), 4)
+    bad = _shape(group_dim=64, R=11, t_cap=1040, n_q_heads=8, n_kv_heads=2)   # 16 | t_cap, 64 does not
+    bad.code_bits = 6
+    assert b.lib.cvq_pack_codes6(ctypes.byref(bad), FAKE, FAKE, None) == 2          # CVQ_ERR_SHAPE
+    narrow = _shape()
+    narrow.code_bits = 6
+    assert b.lib.cvq_pack_codes6(ctypes.byref(narrow), FAKE, FAKE, None) == 4       # UNSUPPORTED
+    odd = _shape(group_dim=64, R=11, t_cap=1024, n_q_heads=8, n_kv_heads=2)
+    odd.code_bits = 7
+    assert b.lib.cvq_pack_codes6(ctypes.byref(odd), FAKE, FAKE, None) == 4
+    unpacked = _shape(group_dim=64, R=11, t_cap=1024, n_q_heads=8, n_kv_heads=2)  # code_bits 0
+    assert b.lib.cvq_pack_codes6(ctypes.byref(unpacked), FAKE, FAKE, None) == 4
+    assert b.lib.cvq_pack_codes6(ctypes.byref(s), None, FAKE, None) == 1             # NULL
+    assert b.lib.cvq_pack_codes6(ctypes.byref(s), FAKE, MISALIGNED, None) == 3       # ALIGN
+    # the decode refuses a packed narrow layout and a packed t_cap off the 64 grid
+    st = b.lib.cvq_decode_attn_gqa(ctypes.byref(narrow), FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, FAKE,
+                                   0, 2, FAKE, FAKE, FAKE, None)
+    assert st == 4
+    st = b.lib.cvq_decode_attn_gqa(ctypes.byref(bad), FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, FAKE,
+                                   0, 2, FAKE, FAKE, FAKE, None)
+    assert st == 2

@@ -75,3 +75,15 @@ def test_roofline_legs_by_hand():
     assert math.isclose(legs["sfu_us"], 4.5353, rel_tol=1e-4)
     assert math.isclose(legs["hbm_us"], 35_651_584 / 6528.7e9 * 1e6, rel_tol=1e-12)
     assert max(legs, key=legs.get) == "fp32_us"
+
+
+def test_packed_code_bytes_by_hand():
+    # the paper's 1-bit setting at 128K tokens: 131072 tokens x 8 KV heads x (key + value)
+    # x 2 groups x 11 rounds = 46,137,344 codes; packed at 6 bits: 34,603,008 bytes (3/4)
+    w = W["llama8b_layer_T131072_R11_g64"]
+    cbs = 2 * 8 * 2 * 11 * 64 * 64 * 4
+    assert bench.code_bytes(w, 131072, 6) == 34_603_008 + cbs
+    assert bench.code_bytes(w, 131072, 8) == 46_137_344 + cbs
+    class A:  # noqa: E701 - stand-in for the parsed arguments
+        code_bits = 0
+    assert bench.code_bits_of(w, A) == 6 and bench.code_bits_of(W["llama8b_layer_T131072_R1"], A) == 8
