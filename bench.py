@@ -391,10 +391,21 @@ def run_gpu(args):
                                 device_id=dev)
 
     w = workloads.WORKLOADS[args.workload]
+    partitioned = args.partition == "heads" and world > 1
+    if partitioned and world > w.n_kv_heads:
+        raise SystemExit(f"--partition heads needs at most {w.n_kv_heads} ranks")
     n_sets = N_INPUT_SETS
     sets = []
     for i in range(n_sets):
         d = workloads.generate(w, layer=i)
+        if partitioned:
+            # this rank's KV heads (and their query heads) of the layer; no data exchange
+            full_q_bits = d.get("q_bits")
+            d, _ = cvq.shard_kv_heads(d, w.n_q_heads, w.n_kv_heads, rank, world)
+            if full_q_bits is not None:
+                g = w.n_q_heads // w.n_kv_heads
+                h0, h1 = cvq.kv_head_range(w.n_kv_heads, rank, world)
+                d["q_bits"] = full_q_bits[:, h0 * g:h1 * g].copy()
         if d["q_dtype"] == "bf16":
             q = torch.from_numpy(d["q_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
         else:
@@ -626,7 +637,9 @@ def run_gpu(args):
         flops = algorithmic_flops(w, total_tokens)
         achieved_tflops = flops / (dec_mean_ms * 1e-3) / 1e12
         bytes_ = code_bytes(w, total_tokens, cbits)
-        value = whole_job_rate(world, total_tokens, ms_per_step)
+        # replicas: every rank decodes the whole layer; partitioned: the ranks together
+        # decode one layer
+        value = whole_job_rate(1 if partitioned else world, total_tokens, ms_per_step)
         result = {
             "metric": METRIC,
             "value": value,
@@ -636,7 +649,7 @@ def run_gpu(args):
             "warmup": args.warmup,
             "ms_per_step": ms_per_step,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if partitioned else "weak",
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic (seeded codebooks, codes and queries; no trained weights)",
@@ -644,7 +657,8 @@ def run_gpu(args):
             "run": {"form": args.form, "n_splits": S,
                     "l2": f"{N_INPUT_SETS} rotating layer input sets of "
                           f"{code_bytes(w, total_tokens, cbits) / 1e6:.0f} MB (> 126 MB L2 in total)",
-                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                    "parallelism": (f"KV heads partitioned over {world} ranks" if partitioned
+                                    else f"replicas x{world}" if world > 1 else "single GPU")},
             "decode_ms": dec_mean_ms,
             "decode_ms_median": statistics.median(dec_ms),
             "step_ms_median": statistics.median(step_ms),
@@ -661,7 +675,8 @@ def run_gpu(args):
                                         f"{SINCOS_PAIRS_PER_CLK} sin+cos pairs and {EXP2_PER_CLK} "
                                         f"exp2 per SM-clock (measured); HBM {pk['hbm_gbs']} GB/s "
                                         f"({pk_src})"},
-            "e2e": {"value": whole_job_rate(world, total_tokens, e2e_ms), "unit": "KV tokens/s per layer",
+            "e2e": {"value": whole_job_rate(1 if partitioned else world, total_tokens, e2e_ms),
+                    "unit": "KV tokens/s per layer",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "smem_floor": smem_summary(w, total_tokens, dec_mean_ms, pk, args.form),
             "gpu_launches": args.steps * launches_per_step,
@@ -731,6 +746,9 @@ def main(argv=None):
                          "combine as two launches; table: the pages' per-query-head table "
                          "form; naive: decode the cache to fp16 then attend (comparison path)")
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--partition", choices=["replicas", "heads"], default="replicas",
+                    help="under torchrun: every rank decodes the whole layer (replicas, weak "
+                         "scaling) or a disjoint slice of its KV heads (heads, strong scaling)")
     ap.add_argument("--code-bits", type=int, choices=[6, 8], default=0,
                     help="stored bits per code: 6 = packed (64-entry codebooks only); "
                          "default 6 for 64-entry codebooks, 8 otherwise")

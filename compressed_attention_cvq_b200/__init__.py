@@ -103,6 +103,40 @@ def pack_codes6(shape, codes, out=None, stream=None):
     return out
 
 
+def kv_head_range(n_kv_heads, rank, world):
+    """The contiguous slice [h0, h1) of KV heads that rank `rank` of `world` decodes when a
+    layer is partitioned by KV head (balanced: the first n_kv_heads % world ranks take one
+    head more).  KV heads are independent units of the decode -- each with its own query
+    heads, codes and codebooks -- so the ranks exchange no data."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank must be in [0, world)")
+    base, extra = divmod(n_kv_heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def shard_kv_heads(inputs, n_q_heads, n_kv_heads, rank, world):
+    """This rank's share of one layer's inputs: every tensor restricted to its KV heads
+    (and their query heads), made contiguous.  `inputs` holds q [B, Hq, 128], key_cb and
+    val_cb [Hkv, ...], key_codes and val_codes [B, Hkv, ...] and seq_lens [B] (torch tensors
+    or numpy arrays); codebooks shared by all heads (leading dim 1) are kept whole.
+    Returns (shard, (h0, h1))."""
+    h0, h1 = kv_head_range(n_kv_heads, rank, world)
+    g = n_q_heads // n_kv_heads
+
+    def contig(x):
+        return x.contiguous() if hasattr(x, "contiguous") else x.copy()
+
+    out = dict(inputs)
+    out["q"] = contig(inputs["q"][:, h0 * g:h1 * g])
+    for k in ("key_cb", "val_cb"):
+        if inputs[k].shape[0] != 1:
+            out[k] = contig(inputs[k][h0:h1])
+    for k in ("key_codes", "val_codes"):
+        out[k] = contig(inputs[k][:, h0:h1])
+    return out, (h0, h1)
+
+
 def split_tokens(shape, n_splits):
     return _b.lib.cvq_split_tokens(ctypes.byref(shape), n_splits)
 
