@@ -29,10 +29,12 @@
 //     touch 32 different banks and never the same address.
 //
 // Tokens: kSlots = 4 per warp per step; slot sigma handles t_begin + sigma + kSlots*j.
-// The phase of a lane's 4 pairs is re-seeded from the exact fixed-point turn every 8
-// steps (every tile at R = 1, every second tile at R = 2) and advances by
-// e^{i theta_j kSlots} per step in between (at most 7 products, rounding error ~1e-7 each).  Code bytes of the
-// next tile are copied to shared memory with cp.async while the current tile computes.
+// The phase of a lane's 4 pairs is re-seeded from the exact fixed-point turn at the start
+// of every tile and advances by e^{i theta_j kSlots} per step within it (at most
+// kSteps - 1 = 7 products at R = 1, 3 at R = 2, rounding error ~1e-7 each).  Each warp
+// copies the code bytes of its own token slots for the next tile to shared memory with
+// cp.async while the current tile computes, so the only barrier of a tile is the cluster
+// barrier of the score exchange.
 #include <cooperative_groups.h>
 
 #include <type_traits>
@@ -65,12 +67,6 @@ struct Cfg {
                                   sizeof(float) * (kBins + kXchg + kWarps * kHeads + 4 * kHeads) +
                                   kCodeBytes + 16;   // + the TMA mbarrier
   static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
-  // the RoPE phase is re-seeded exactly every kReseedSteps steps (every tile at R = 1, every
-  // second tile at R = 2), so at most kReseedSteps - 1 recurrence products separate a phase
-  // from its exact seed
-  static constexpr int kReseedSteps = 8;
-  static constexpr int kReseedTiles = kReseedSteps / kSteps;
-  static_assert(kReseedTiles * kSteps == kReseedSteps, "whole tiles between seeds");
 };
 
 __device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
@@ -159,9 +155,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
 
   const size_t code_row = (static_cast<size_t>(b) * a.n_kv_heads + h) * a.t_cap;
   // copy the code bytes of this CTA's 8 groups for one tile (key and value, every round)
+  // each warp copies the code bytes of its own token slots (sigma = 4 warp + tau over the
+  // tile's steps), so only the warp's own copies must land before it reads them: no
+  // CTA-wide barrier per tile for the codes
   auto stage_codes = [&](int t_tile, int buf) {
-    for (int i = tid; i < kTile * R; i += C::kThreads) {
-      const int tt = i % kTile, r = i / kTile;
+    static_assert(C::kSteps * 4 * R == 32, "one (token, round) per lane and tile");
+    {
+      const int r = lane % R, slot = (lane / R) & 3, st = lane / (4 * R);
+      const int tt = st * C::kSlots + warp * 4 + slot;
       const int t = t_tile + tt;
       if (t < t_end && in_bounds(a.fault, t, a.t_cap) &&
           in_bounds(a.fault, ((buf * kTile + tt) * R + r) * 16 + 15, C::kCodeBytes)) {
@@ -206,8 +207,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
                              load_q(a.q, a.q_dtype, qb + 2 * pp + 1) * qscale);
     }
   }
-  // phase of the lane's pairs: re-seeded from the exact turn every kReseedSteps steps,
-  // advanced by e^{i theta kSlots} per step in between
+  // phase of the lane's pairs: re-seeded from the exact turn at the first token of every
+  // tile, advanced by e^{i theta kSlots} per step within the tile
   float2 ph[4], adv[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) adv[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], C::kSlots);
@@ -305,10 +306,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     float* xb = xchg + buf * (kTile * kHeads);
     float* pxb = peer_xchg + buf * (kTile * kHeads);
 
-    if (tile % C::kReseedTiles == 0) {   // exact seed at least every kReseedSteps steps
 #pragma unroll
-      for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
-    }
+    for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
     float s_part[C::kSteps];
     constexpr int kGS = C::kSteps >= 4 ? 4 : C::kSteps;   // steps per pass group
 #pragma unroll
@@ -408,8 +407,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     const int t_tile = t_begin + tile * kTile;
     const int buf = tile & 1;
     if (tile > 0) {
-      cp_async_wait_all();      // this tile's codes (issued one tile ago) have landed
-      __syncthreads();          // ... for every thread; the other buffer is free again
+      cp_async_wait_all();      // this warp's codes of this tile (issued one tile ago) landed
+      __syncwarp();             // ... for every lane; the warp is done with the other buffer
     }
     if (tile + 1 < n_tiles) stage_codes(t_tile + kTile, buf ^ 1);
     if (t_tile + kTile <= t_end) {
