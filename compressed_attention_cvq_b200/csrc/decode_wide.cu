@@ -95,12 +95,8 @@ __device__ __forceinline__ void stage_codebook(float4* dst, const float* src, in
   if (lane < rc) bulk_load(dst + lane * kWideCodes * kWChunks, src + lane * kWideCodes * 4 * kWChunks, kRound, bar);
 }
 
-// kFullSlice: the round loops of the token steps run over exactly kRC rounds, with no
-// per-round bound check.  A CTA whose slice has fewer rounds (rc_act < kRC; used when every
-// slice has at least 10, e.g. R = 21 = 11 + 10) pads it with all-zero rounds: zeroed
-// codewords and code 0, so the key sums and the bins of the real rounds are unchanged, and
-// the epilogue reads only the real rounds.  The CTAs of a cluster meet at a barrier every
-// tile, so the padded CTA only fills time it spent waiting for its 11-round peer.
+// kFullSlice: every CTA of the cluster holds exactly kRC rounds (R a multiple of 11), so the
+// round loops run without a per-round bound check
 template <bool kFullSlice>
 __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeArgs a, int R) {
   extern __shared__ __align__(128) float4 smem4[];
@@ -123,8 +119,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   const int n_slices = C >> 1;
   const int RCeil = (R + n_slices - 1) / n_slices;
   const int r0 = rs * RCeil;
-  const int rc_act = min(R, r0 + RCeil) - r0;     // this CTA's real rounds
-  const int rc = kFullSlice ? kRC : rc_act;        // rounds of the token-step loops
+  const int rc = kFullSlice ? kRC : min(R, r0 + RCeil) - r0;
 
   const int split = blockIdx.x / C;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -162,12 +157,12 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   const size_t row_bytes = packed6 ? static_cast<size_t>(a.t_cap) / 4 * 3 : static_cast<size_t>(a.t_cap);
   constexpr int kChunksPerRow = kWTile / 16;           // unpacked; packed uses 3/4 of them
   auto stage_codes = [&](int t_tile, int buf) {
-    const int n = 2 * rc_act * kChunksPerRow;
+    const int n = 2 * rc * kChunksPerRow;
     const size_t tile_byte = packed6 ? static_cast<size_t>(t_tile) / 4 * 3 : static_cast<size_t>(t_tile);
     const int need = packed6 ? ((t_end - t_tile) * 3 + 3) / 4 : (t_end - t_tile);   // bytes with tokens < t_end
     for (int i = tid; i < n; i += kWThreads) {
-      const int kind = i / (rc_act * kChunksPerRow);
-      const int r = (i / kChunksPerRow) % rc_act;
+      const int kind = i / (rc * kChunksPerRow);
+      const int r = (i / kChunksPerRow) % rc;
       const int q16 = i % kChunksPerRow;
       if (16 * q16 < need && in_bounds(a.fault, tile_byte + 16 * q16 + 15, row_bytes)) {
         const uint8_t* src = (kind ? a.val_codes : a.key_codes) + (code_row0 + r) * row_bytes + tile_byte + 16 * q16;
@@ -181,11 +176,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   const float* vcb = a.val_cb + h * a.val_cb_stride +
                      (static_cast<size_t>(G) * R + r0) * kWideCodes * kWideVDims;
   if (tid == 0) mbar_init(tma_bar, 1);
-  if (warp == 0) stage_codebook(cw_s, kcb, rc_act, tma_bar);
-  // padded rounds: zero codewords (rounds rc_act .. rc - 1 of cw_s; the TMA writes only
-  // the real rounds), visible to every thread after the first tile's barrier
-  for (int i = rc_act * kWideCodes * kWChunks + tid; i < rc * kWideCodes * kWChunks; i += kWThreads)
-    cw_s[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) stage_codebook(cw_s, kcb, rc, tma_bar);
   stage_codes(t_begin, 0);
   cp_async_commit();
   for (int i = tid; i < kWideCodes * kBinStride / 4; i += kWThreads)
@@ -244,7 +235,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
       const uint8_t* srow = code_s + (buf * 2 + kind) * kRC * kWTile;     // packed rows
 #pragma unroll
       for (int r = 0; r < kRC; ++r)
-        if (r < rc_act) {                  // padded rounds keep code 0
+        if (r < rc) {
           const uint32_t c = packed6 ? static_cast<uint32_t>(packed6_code(srow + r * kWTile, t))
                                      : static_cast<uint32_t>(src[r * kWTile]);
           wv[r >> 2] |= c << (8 * (r & 3));
@@ -381,13 +372,13 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   // them before the TMA writes)
   if (warp == 0) {
     fence_proxy_async_smem();
-    stage_codebook(cw_s, vcb, rc_act, tma_bar);
+    stage_codebook(cw_s, vcb, rc, tma_bar);
   }
   if (!mbar_wait(tma_bar, 1) && tid == 0) atomicOr(a.fault, kFaultCopyTimeout);
   const float* cv = reinterpret_cast<const float*>(cw_s);
   const int eh = (tid >> 6) & 3, ed = tid & 63, half = tid >> 8;
   float o = 0.f;
-  for (int r = 0; r < rc_act; ++r) {
+  for (int r = 0; r < rc; ++r) {
     const float* br = bins + 4 * r + eh;
     const float* vr = cv + static_cast<size_t>(r) * kWideCodes * kWideVDims + ed;
 #pragma unroll 8
@@ -439,12 +430,8 @@ cudaError_t launch_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t st
 }  // namespace
 
 cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
-  // the token-step loops run over 11 rounds when every round slice has at least 10 real
-  // ones (R = 10, 11, 20, 21, 22), padding a shorter slice with zero rounds
-  const int n_slices = wide_round_slices(s.R);
-  const int per = (s.R + n_slices - 1) / n_slices;
-  const int min_rc = s.R - (n_slices - 1) * per;
-  return min_rc >= kRC - 1 ? launch_wide<true>(s, a, stream) : launch_wide<false>(s, a, stream);
+  // R = 11 or 22: every round slice is a full 11 rounds
+  return s.R % kRC == 0 ? launch_wide<true>(s, a, stream) : launch_wide<false>(s, a, stream);
 }
 
 }  // namespace cvq
