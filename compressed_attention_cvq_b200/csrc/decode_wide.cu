@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   float* red_l = red_m + kWWarps * kWHeads;                                   // [16][4]
   float* mref_s = red_l + kWWarps * kWHeads;                                  // [4]
   float* l_s = mref_s + kWHeads;                                              // [4]
-  float* fac_s = l_s + kWHeads;                                               // [4]
+  float* fac_s = l_s + kWHeads;                                               // [4] spare
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(fac_s + kWHeads);           // codebook copies
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -181,11 +181,9 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   cp_async_commit();
   for (int i = tid; i < kWideCodes * kBinStride / 4; i += kWThreads)
     reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (tid < kWHeads) {
-    mref_s[tid] = -INFINITY;
-    l_s[tid] = 0.f;
-  }
-  for (int i = tid; i < kWWarps * kWHeads; i += kWThreads) red_l[i] = 0.f;
+  // softmax state of head tid & 3, held by every thread: the reference max (the same in
+  // every thread of the CTA) and this thread's share of l
+  float m_ref = -INFINITY, l_acc = 0.f;
 
   // this lane's 4 pairs: local pairs 2k, 2k+1 (chunk k) and 2k+16, 2k+17 (chunk 8+k)
   int jp[4];
@@ -312,33 +310,32 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     if (lane < kWHeads) red_m[warp * kWHeads + lane] = mx;
     __syncthreads();
-    if (tid < kWHeads) {
-      float tm = -INFINITY, pend = 0.f;
-      for (int w = 0; w < kWWarps; ++w) {
-        tm = fmaxf(tm, red_m[w * kWHeads + tid]);
-        pend += red_l[w * kWHeads + tid];    // the previous tile's weights
+    // every warp reduces the 16 warps' maxima itself (entry w * 4 + head): lane l takes
+    // entries l and l + 32, then the lanes of its head; every thread ends with the same
+    // tile max of head hh, so the decisions below are the same in every warp
+    float tm = fmaxf(red_m[lane], red_m[lane + 32]);
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+    const bool raise = tm > m_ref + kWSlack;
+    if (__any_sync(0xffffffffu, raise)) {
+      const float m_new = raise ? tm : m_ref;
+      const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
+      const bool rescale = __any_sync(0xffffffffu, m_ref != -INFINITY);
+      l_acc *= f;
+      m_ref = m_new;
+      if (rescale) {   // every earlier atomic was issued before this tile's barriers
+        const float f0 = __shfl_sync(0xffffffffu, f, 0), f1 = __shfl_sync(0xffffffffu, f, 1);
+        const float f2 = __shfl_sync(0xffffffffu, f, 2), f3 = __shfl_sync(0xffffffffu, f, 3);
+        for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) {
+          const int e = i & 3;
+          bins[i] *= e == 0 ? f0 : (e == 1 ? f1 : (e == 2 ? f2 : f3));
+        }
+        __syncthreads();
       }
-      const float mo = mref_s[tid];
-      float f = 1.f;
-      if (tm > mo + kWSlack) {
-        f = (mo == -INFINITY) ? 0.f : exp2f(mo - tm);
-        mref_s[tid] = tm;
-      }
-      l_s[tid] = (l_s[tid] + pend) * f;
-      fac_s[tid] = f;
     }
-    __syncthreads();
-    if (fac_s[0] != 1.f || fac_s[1] != 1.f || fac_s[2] != 1.f || fac_s[3] != 1.f) {
-      for (int i = tid; i < kWideCodes * kBinStride; i += kWThreads) bins[i] *= fac_s[i & 3];
-      __syncthreads();
-    }
-    const float m = mref_s[hh];
-    const float wA = exp2f(sA - m), wB = exp2f(sB - m);
-    float ls = wA + wB;
-    ls += __shfl_xor_sync(0xffffffffu, ls, 4);
-    ls += __shfl_xor_sync(0xffffffffu, ls, 8);
-    ls += __shfl_xor_sync(0xffffffffu, ls, 16);
-    if (lane < kWHeads) red_l[warp * kWHeads + lane] = ls;
+    const float wA = exp2f(sA - m_ref), wB = exp2f(sB - m_ref);
+    l_acc += wA + wB;
     // value reorder: the weight goes to the bin of the token's value code, per own round
     // token slot j of the warp starts at round j (mod rc), so each atomic instruction's 8
     // tokens bin 8 different rounds
@@ -360,11 +357,17 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
     if (wA > 0.f) bin_token(tA, wA);
     if (wB > 0.f) bin_token(tB, wB);
   }
+  // l per head: over the warp's lanes of the head, then over the 16 warps
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 4);
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 8);
+  l_acc += __shfl_xor_sync(0xffffffffu, l_acc, 16);
+  if (lane < kWHeads) red_l[warp * kWHeads + lane] = l_acc;
   __syncthreads();
   if (tid < kWHeads) {
-    float pend = 0.f;
-    for (int w = 0; w < kWWarps; ++w) pend += red_l[w * kWHeads + tid];
-    l_s[tid] += pend;
+    float l = 0.f;
+    for (int w = 0; w < kWWarps; ++w) l += red_l[w * kWHeads + tid];
+    l_s[tid] = l;
+    mref_s[tid] = m_ref;                   // thread tid < 4: head tid
   }
 
   // ---- epilogue: o = bins x value codewords of the own rounds ----

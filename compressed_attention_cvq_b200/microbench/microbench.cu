@@ -171,7 +171,8 @@ __global__ void shfl_kernel(float* out, int iters) {
 // Explicit shared reductions and plain read-modify-write, each lane on its own bank
 // (mode 0: f32, 1: u32, 2: u64 (8-byte aligned, lanes on distinct 8-byte slots),
 //  3: plain ld/add/st f32, 4: plain float4 ld/add/st conflict-free, 5: float4 gather
-//  + two f32 reductions per iteration (mixed))
+//  + two f32 reductions per iteration (mixed), 6: red.shared::cluster.add.f32 on this CTA's
+//  own shared memory (the distributed-shared-memory form of the reduction))
 __global__ void rmw_kernel(float* out, int iters, int mode) {
   __shared__ float4 buf[2048];
   float* bf = reinterpret_cast<float*>(buf);
@@ -198,6 +199,9 @@ __global__ void rmw_kernel(float* out, int iters, int mode) {
         // each warp owns a private 32-float slice per round, so no two threads race
         float* p = bf + ((warp * 8 + r) & 255) * 32 + lane;
         *p += 1.0f;
+      } else if (mode == 6) {
+        unsigned a = (unsigned)__cvta_generic_to_shared(bf + idx);
+        asm volatile("red.shared::cluster.add.f32 [%0], %1;" :: "r"(a), "f"(1.0f) : "memory");
       } else if (mode == 4) {
         float4* p = buf + (((warp * 8 + r) & 63) * 32 + lane);
         float4 v = *p;
@@ -266,6 +270,8 @@ MB_API double cvqmb_run(int kind, int blocks, int threads, int iters, float* out
     case 9: shfl_kernel<<<blocks, threads, 0, s>>>(out, iters); per = 32.0 * iters; break;
     case 10: case 11: case 12: case 13: case 14: case 15:
       rmw_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 10); per = 8.0 * iters; break;
+    case 19:
+      rmw_kernel<<<blocks, threads, 0, s>>>(out, iters, 6); per = 8.0 * iters; break;
     case 16: case 17: case 18:
       gred_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 16); per = 8.0 * iters; break;
     default: return -1;
