@@ -23,9 +23,11 @@ KINDS = {0: "ffma", 1: "ffma2 (f32x2, 2 FMA each)", 2: "sincos (__sincosf)", 3: 
          16: "red.global.add.v4.f32 random (L2, 64 KB per CTA)",
          17: "red.global.add.f32 random (L2, 64 KB per CTA)",
          18: "red.global.add.v4.f32, 25% on 4 hot slots",
-         19: "red.shared::cluster.add.f32 distinct (own CTA)"}
+         19: "red.shared::cluster.add.f32 distinct (own CTA)",
+         20: "warp-owned float4 bins, ld/add/st, equal codes take turns (uniform codes)",
+         21: "warp-owned float4 bins, ld/add/st, equal codes take turns (25% code 0)"}
 ITERS = {0: 4000, 1: 2000, 2: 1000, 3: 1000, 4: 4000, 5: 4000, 6: 2000, 7: 2000, 8: 500, 9: 2000, 10: 2000, 11: 2000, 12: 2000, 13: 2000, 14: 2000, 15: 2000,
-         16: 200, 17: 200, 18: 100, 19: 2000}
+         16: 200, 17: 200, 18: 100, 19: 2000, 20: 500, 21: 500}
 GLOBAL_KINDS = (16, 17, 18)     # take a scratch buffer of blocks x 16384 floats
 
 

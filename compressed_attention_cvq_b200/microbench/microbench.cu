@@ -244,12 +244,62 @@ __global__ void gred_kernel(float* buf, int iters, int mode) {
   }
 }
 
+// Value bins owned by one warp, updated without atomics (one 16-byte read-add-write adds a
+// token's weights of 4 heads to the bin of its code): each warp owns 64 float4 bins, each
+// lane takes one (token, group) per operation -- its code byte and its 4 weights from
+// shared memory -- and lanes holding the same code take turns (__match_any_sync, rank
+// among equal codes, one pass per rank, __syncwarp between passes).  skew = 0: codes
+// uniform over 64; skew = 1: a quarter of them 0 (a hot code).  One op = one (token, group)
+// update of 4 heads.  Indexes: bins (warp & 31) * 64 + code < 2048, weights < 256, codes
+// < 8192.
+__global__ void owned_bins_kernel(float* out, int iters, int skew) {
+  __shared__ float4 bins[2048];
+  __shared__ float4 wts[256];
+  __shared__ uint8_t codes[8192];
+  unsigned x = 2654435761u * (threadIdx.x + 1) + 97u * blockIdx.x;
+  for (int i = threadIdx.x; i < 2048; i += blockDim.x) bins[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) wts[i] = make_float4(1.f, 0.5f, 0.25f, 0.125f);
+  for (int i = threadIdx.x; i < 8192; i += blockDim.x) {
+    x = x * 1664525u + 1013904223u;
+    int c = static_cast<int>(x >> 26);
+    if (skew && ((x >> 20) & 3u) == 0u) c = 0;
+    codes[i] = static_cast<uint8_t>(c);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  float4* mine = bins + ((threadIdx.x >> 5) & 31) * 64;
+  const unsigned below = (1u << lane) - 1u;
+  int pos = (threadIdx.x >> 5) * 32 + lane;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      pos = (pos + 32 * 9) & 8191;
+      const int c = codes[pos] & 63;
+      const float4 w = wts[pos & 255];
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(peers & below);
+      const int passes = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(rank));
+      for (int k = 0; k <= passes; ++k) {
+        if (rank == k) {
+          float4 v = mine[c];
+          v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+          mine[c] = v;
+        }
+        __syncwarp();
+      }
+    }
+  }
+  __syncthreads();
+  if (bins[threadIdx.x & 2047].x == 123.456f) out[threadIdx.x] = 1.f;
+}
+
 }  // namespace
 
 // kind: 0 ffma, 1 ffma2, 2 sincos, 3 exp2, 4 lds128 conflict-free, 5 lds128 random,
 //       6 atomic distinct banks, 7 atomic random, 8 atomic same address, 9 shfl,
 //       10..15 rmw_kernel modes 0..5 (mode 5 counts one gather + two reductions as one op),
-//       16..18 gred_kernel modes 0..2 (`out` must hold blocks x 16384 floats)
+//       16..18 gred_kernel modes 0..2 (`out` must hold blocks x 16384 floats),
+//       19 rmw_kernel mode 6, 20..21 owned_bins_kernel skew 0..1 (blockDim <= 1024)
 // Returns the operation count of the launch (per-thread ops x threads x blocks), or
 // -1 for an unknown kind / launch error.  Operations: FMA lanes (ffma2 counts 2 per
 // instruction), sin+cos pairs, exp2, 16-byte loads, atomics, shuffles.
@@ -272,6 +322,9 @@ MB_API double cvqmb_run(int kind, int blocks, int threads, int iters, float* out
       rmw_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 10); per = 8.0 * iters; break;
     case 19:
       rmw_kernel<<<blocks, threads, 0, s>>>(out, iters, 6); per = 8.0 * iters; break;
+    case 20: case 21:
+      if (threads > 1024) return -1;
+      owned_bins_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 20); per = 8.0 * iters; break;
     case 16: case 17: case 18:
       gred_kernel<<<blocks, threads, 0, s>>>(out, iters, kind - 16); per = 8.0 * iters; break;
     default: return -1;

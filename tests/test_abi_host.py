@@ -337,3 +337,21 @@ def test_packed_code_layout_validation():
     st = b.lib.cvq_decode_attn_gqa(ctypes.byref(bad), FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, FAKE,
                                    0, 2, FAKE, FAKE, FAKE, None)
     assert st == 2
+
+
+def test_c_attend_loop_compiles(tmp_path):
+    """The C driver of cvq_attend (tests/c_abi/attend_loop.c) builds with -Wall -Wextra
+    -Werror against cvq.h, libcvq.so and the CUDA runtime; without a GPU it reports the CUDA
+    error and exits non-zero instead of crashing."""
+    import subprocess
+    import sys
+
+    sys.path.insert(0, os.path.join(ROOT, "tests", "c_abi"))
+    import build_attend_loop
+
+    try:
+        exe = build_attend_loop.build(str(tmp_path / "attend_loop"))
+    except RuntimeError as e:
+        pytest.skip(str(e))
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 1 and "usage" in r.stderr

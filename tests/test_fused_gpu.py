@@ -103,3 +103,25 @@ def test_128k_layer_with_one_and_two_splits():
         torch.cuda.synchronize()
         assert_close(out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
                      ref_out, ref_lse, heads=heads)
+
+
+def test_rope_base_change_between_calls():
+    """The library keeps the phase increments of the last RoPE base a thread asked for: calls
+    that alternate between two bases (500000 and 10000) each match the oracle run with their
+    own base."""
+    lens = [1200, 777]
+    cases = {base: _case_base(base, lens) for base in (500000.0, 10000.0)}
+    for base in (500000.0, 10000.0, 500000.0, 10000.0):
+        d, dd = cases[base]
+        out, lse = cvq.attend(dd["q"], dd["key_cb"], dd["val_cb"], dd["key_codes"], dd["val_codes"],
+                              dd["seq_lens"], base, n_splits=3)
+        torch.cuda.synchronize()
+        ref_out, ref_lse = run_oracle(d)
+        assert_close(out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                     ref_out, ref_lse)
+
+
+def _case_base(base, lens):
+    d = workloads.small(batch=len(lens), n_q_heads=8, n_kv_heads=2, t_cap=1280, R=1,
+                        seq_lens=np.asarray(lens, np.int32), seed=97, rope_base=base)
+    return d, to_device(d)
