@@ -161,24 +161,8 @@ cvq_status decode_gqa_impl(const cvq_shape* s, const void* q, int q_dtype, const
 
 namespace cvq {
 
-// The turns depend on rope_base alone, and a decode loop passes the same base at every
-// step, while the 64 long-double powers cost ~20 us of host time: each calling thread keeps
-// the turns of the last base it asked for.
-void phase_turns_host(float rope_base, PhaseTurns* out) {
-  thread_local bool have = false;
-  thread_local uint32_t have_bits = 0;
-  thread_local PhaseTurns have_turns;
-  uint32_t bits;
-  std::memcpy(&bits, &rope_base, sizeof(bits));
-  if (!have || bits != have_bits) {
-    phase_turns_exact(rope_base, &have_turns);
-    have_bits = bits;
-    have = true;
-  }
-  *out = have_turns;
-}
-
-void phase_turns_exact(float rope_base, PhaseTurns* out) {
+// F_j for every pair, computed in long double
+static void phase_turns_exact(float rope_base, PhaseTurns* out) {
   const long double two_pi = 6.283185307179586476925286766559L;
   const long double base = static_cast<long double>(rope_base);
   for (int j = 0; j < kPairs; ++j) {
@@ -194,6 +178,23 @@ void phase_turns_exact(float rope_base, PhaseTurns* out) {
     }
     out->F[j] = f;
   }
+}
+
+// The turns depend on rope_base alone, and a decode loop passes the same base at every
+// step, while the 64 long-double powers cost ~20 us of host time: each calling thread keeps
+// the turns of the last base it asked for.
+void phase_turns_host(float rope_base, PhaseTurns* out) {
+  thread_local bool have = false;
+  thread_local uint32_t have_bits = 0;
+  thread_local PhaseTurns have_turns;
+  uint32_t bits;
+  std::memcpy(&bits, &rope_base, sizeof(bits));
+  if (!have || bits != have_bits) {
+    phase_turns_exact(rope_base, &have_turns);
+    have_bits = bits;
+    have = true;
+  }
+  *out = have_turns;
 }
 
 cvq_status attend_into(const cvq_shape* s, const void* q, int q_dtype, const float* key_cb,

@@ -45,10 +45,7 @@ struct PhaseTurns {
   unsigned long long F[kPairs];
 };
 
-// Host: fill F_j for a RoPE base (long double for the 64-bit fraction).  phase_turns_exact
-// computes them; phase_turns_host returns the calling thread's copy for the last base it
-// asked for, recomputing only when the base changes.
-void phase_turns_exact(float rope_base, PhaseTurns* out);
+// Host: fill F_j for a RoPE base (long double for the 64-bit fraction).
 void phase_turns_host(float rope_base, PhaseTurns* out);
 
 // cos/sin of 2 pi * (turn64 / 2^64); the top 32 bits give the angle to 2^-32 turns,
