@@ -95,10 +95,10 @@ __device__ __forceinline__ void stage_codebook(float4* dst, const float* src, in
   if (lane < rc) bulk_load(dst + lane * kWideCodes * kWChunks, src + lane * kWideCodes * 4 * kWChunks, kRound, bar);
 }
 
-// kFullSlice: every CTA of the cluster holds exactly kRC rounds (R a multiple of 11), so the
-// round loops run without a per-round bound check
-template <bool kFullSlice>
-__global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeArgs a, int R) {
+// One CTA's work.  kRounds > 0: the CTA's round slice holds exactly kRounds rounds, so the
+// round loops run without a per-round bound check; 0: the slice size is computed at run time.
+template <int kRounds>
+__device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
   extern __shared__ __align__(128) float4 smem4[];
   float4* cw_s = smem4;                                                       // codewords
   float* bins = reinterpret_cast<float*>(smem4 + kRC * kWideCodes * kWChunks);
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   const int n_slices = C >> 1;
   const int RCeil = (R + n_slices - 1) / n_slices;
   const int r0 = rs * RCeil;
-  const int rc = kFullSlice ? kRC : min(R, r0 + RCeil) - r0;
+  const int rc = kRounds > 0 ? kRounds : min(R, r0 + RCeil) - r0;
 
   const int split = blockIdx.x / C;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -409,11 +409,23 @@ __global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const DecodeA
   if (a.counters != nullptr) merge_tail(a, b, h, hq0, kWHeads, C * a.n_splits);
 }
 
-template <bool kFullSlice>
+// kFirst / kRest: the rounds of the first round slice / of the others, known when the kernel
+// is compiled (0: computed at run time).  Every CTA of a cluster meets the same barriers
+// whichever body it runs.
+template <int kFirst, int kRest>
+__global__ void __launch_bounds__(kWThreads, 1) decode_wide_kernel(const __grid_constant__ DecodeArgs a, int R) {
+  if (kFirst == kRest || (cg::this_cluster().block_rank() >> 1) == 0) {
+    wide_body<kFirst>(a, R);
+  } else {
+    wide_body<kRest>(a, R);
+  }
+}
+
+template <int kFirst, int kRest>
 cudaError_t launch_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
   const int C = wide_cluster_size(s.R);
   static PerDeviceFlag smem_set;
-  cudaError_t e = set_smem_limit_once(smem_set, decode_wide_kernel<kFullSlice>, kWSmem);
+  cudaError_t e = set_smem_limit_once(smem_set, decode_wide_kernel<kFirst, kRest>, kWSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.n_splits * C), s.n_kv_heads, s.batch);
@@ -427,14 +439,16 @@ cudaError_t launch_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_wide_kernel<kFullSlice>, a, s.R);
+  return cudaLaunchKernelEx(&cfg, decode_wide_kernel<kFirst, kRest>, a, s.R);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_wide(const cvq_shape& s, const DecodeArgs& a, cudaStream_t stream) {
-  // R = 11 or 22: every round slice is a full 11 rounds
-  return s.R % kRC == 0 ? launch_wide<true>(s, a, stream) : launch_wide<false>(s, a, stream);
+  // R = 11 or 22: every round slice is 11 rounds; R = 21: slices of 11 and 10 rounds
+  if (s.R % kRC == 0) return launch_wide<kRC, kRC>(s, a, stream);
+  if (s.R == 2 * kRC - 1) return launch_wide<kRC, kRC - 1>(s, a, stream);
+  return launch_wide<0, 0>(s, a, stream);
 }
 
 }  // namespace cvq
