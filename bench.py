@@ -328,6 +328,57 @@ def oracle_sample(w: workloads.Workload, budget_s: float = 12.0, layer: int = 0)
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def serving_loop(w, dset, shape, S, ws, out, lse, stream, dev, n_steps=50):
+    """The decode step as a serving loop runs it: the code cache and codebooks stay resident
+    on the device (they are state, not per-step inputs); every step copies the new token's
+    query, key, value and cache position from pinned host memory, appends the new codes
+    (cvq_encode_append, at the last position of every sequence so the cache keeps its
+    length), attends (cvq_attend), copies out and lse to pinned host memory and waits for
+    them, as a sampler must before the next step.  Device-timed with events around the
+    steps, so host enqueue time and the per-step wait are inside the measurement."""
+    h = dset["host"]
+    nk, nv = workloads.new_tokens(w, layer=0)
+    if h["q_dtype"] == "bf16":
+        hq = torch.from_numpy(h["q_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    else:
+        hq = torch.from_numpy(h["q"]).pin_memory()
+    hk = torch.from_numpy(nk).pin_memory()
+    hv = torch.from_numpy(nv).pin_memory()
+    hpos = torch.from_numpy(np.maximum(h["seq_lens"] - 1, 0).astype(np.int32)).pin_memory()
+    dq, dk, dv, dpos = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hpos))
+    ho = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+    hl = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dpos.copy_(hpos, non_blocking=True)
+        cvq.encode_append(shape, dk, dv, dset["key_cb"], dset["val_cb"], dpos, dset["key_codes"],
+                          dset["val_codes"])
+        o, l = cvq.attend_fused(shape, dq, dset["key_cb"], dset["key_codes"], dset["val_codes"],
+                                dset["seq_lens"], dset["val_cb"], S, workspace=ws, out=out, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(5):
+        one()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hpos))
+    d2h = ho.numel() * 4 + hl.numel() * 4
+    return {"ms_per_step": e0.elapsed_time(e1) / n_steps, "steps": n_steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "launches_per_step": 2,
+            "what": "cache resident; per step: new token's q, k, v, position in; append + attend; "
+                    "out, lse back and waited for"}
+
+
 def sustained_run(step, args, n_sets, stream, dev):
     """Replay a CUDA graph of n_sets consecutive steps until about SUSTAINED_S seconds of
     device time have passed; per-step device time from one event pair per replay."""
@@ -621,6 +672,11 @@ def run_gpu(args):
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / n_e2e, dev)
+    serving = None if (partitioned or args.form != "gqa") else serving_loop(w, sets[0], shape, S, ws,
+                                                                          out, lse, stream, dev)
+    if serving is not None:
+        serving["ms_per_step"] = max_over_ranks(serving["ms_per_step"], dev)
+
     fault = cvq.fault_status(clear=True)     # a bounded codebook-copy wait gave up: invalid run
     if fault:
         raise RuntimeError(f"device fault word {fault:#x} after the timed steps")
@@ -678,6 +734,9 @@ def run_gpu(args):
             "e2e": {"value": whole_job_rate(1 if partitioned else world, total_tokens, e2e_ms),
                     "unit": "KV tokens/s per layer",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e_serving": None if serving is None else dict(
+                serving, value=whole_job_rate(world, total_tokens, serving["ms_per_step"]),
+                unit="KV tokens/s per layer"),
             "smem_floor": smem_summary(w, total_tokens, dec_mean_ms, pk, args.form),
             "gpu_launches": args.steps * launches_per_step,
             "sustained": sustained,
