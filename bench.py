@@ -336,6 +336,10 @@ def serving_loop(w, dset, shape, S, ws, out, lse, stream, dev, n_steps=50):
     length), attends (cvq_attend), copies out and lse to pinned host memory and waits for
     them, as a sampler must before the next step.  Device-timed with events around the
     steps, so host enqueue time and the per-step wait are inside the measurement."""
+    import torch
+
+    import compressed_attention_cvq_b200 as cvq
+
     h = dset["host"]
     nk, nv = workloads.new_tokens(w, layer=0)
     if h["q_dtype"] == "bf16":

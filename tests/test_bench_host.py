@@ -5,6 +5,7 @@ value worked out by hand from the definitions in the docstrings (per token and q
 (group, round); per token and KV head: one code byte per (group, round) for keys and for
 values)."""
 import math
+import os
 
 import pytest
 
@@ -87,3 +88,45 @@ def test_packed_code_bytes_by_hand():
     class A:  # noqa: E701 - stand-in for the parsed arguments
         code_bits = 0
     assert bench.code_bits_of(w, A) == 6 and bench.code_bits_of(W["llama8b_layer_T131072_R1"], A) == 8
+
+
+def _unresolved_globals(path):
+    """Names that a function of the file reads as globals but that neither the module
+    defines (assignment, import, def, class) nor Python provides (builtins)."""
+    import builtins
+    import symtable
+
+    src = open(path).read()
+    top = symtable.symtable(src, path, "exec")
+    defined = {s.get_name() for s in top.get_symbols()
+               if s.is_assigned() or s.is_imported() or s.is_namespace()}
+    known = defined | set(dir(builtins)) | {"__file__", "__name__"}
+    bad = []
+
+    def walk(t):
+        for ch in t.get_children():
+            for s in ch.get_symbols():
+                if s.is_referenced() and s.is_global() and s.get_name() not in known:
+                    bad.append(f"{ch.get_name()}: {s.get_name()}")
+            walk(ch)
+
+    walk(top)
+    return bad
+
+
+def _python_sources():
+    import glob
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = []
+    for sub in ("*.py", "compressed_attention_cvq_b200/**/*.py", "oracle/*.py", "tests/**/*.py"):
+        out += [os.path.relpath(p, root) for p in glob.glob(os.path.join(root, sub), recursive=True)]
+    return sorted(out)
+
+
+@pytest.mark.parametrize("rel", _python_sources())
+def test_every_global_name_resolves(rel):
+    """A function that reads a name its module never binds (a missing import) fails only
+    when that function runs, on the GPU machine for most of these files: check statically."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    assert _unresolved_globals(os.path.join(root, rel)) == []
