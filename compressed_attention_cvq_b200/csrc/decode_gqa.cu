@@ -241,7 +241,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   // mslot) -> full scores and the warp's maxima of tile t into mslot -> raise the reference
   // max from tile t-1's maximum if needed -> weights and bin atomics of tile t-1 (scores and
   // value codes kept in registers for one iteration).  The only barrier of a tile is the
-  // cluster barrier (plus the code-copy barrier at its start); no CTA-wide max reduction.
+  // cluster barrier (each warp waits only for its own code copies); no CTA-wide max
+  // reduction.
   float sp[C::kSteps];           // scores of the previous tile's tokens (head hk; -inf = none)
   uint32_t vw[C::kSteps][R];     // value code bytes of those tokens (groups 4 gh .. 4 gh + 3)
 #pragma unroll
