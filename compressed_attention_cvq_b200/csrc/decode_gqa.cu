@@ -65,7 +65,8 @@ struct Cfg {
   static constexpr int kCodeBytes = 2 * kTile * R * 16;               // 2 buffers x (key 8 B + val 8 B) x R
   static constexpr size_t kSmem = sizeof(float4) * kCodeChunks +
                                   sizeof(float) * (kBins + kXchg + kWarps * kHeads + 4 * kHeads) +
-                                  kCodeBytes + 16;   // + the TMA mbarrier
+                                  kCodeBytes + 16 +   // + the TMA mbarrier
+                                  sizeof(unsigned long long) * 4 * kLocalGroups;   // phase turns
   static_assert(kSteps * kSlots == kTile, "tile must be a whole number of steps");
 };
 
@@ -115,6 +116,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   int* mslot = reinterpret_cast<int*>(fh + kHeads);                   // [3][4] tile maxima (ord)
   uint8_t* code_s = reinterpret_cast<uint8_t*>(mslot + 3 * kHeads);   // [2][kTile][R][key 8 | val 8]
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(code_s + C::kCodeBytes);   // codebook copies
+  // F_j of the CTA's 32 pairs (local group k: pairs 4 k .. 4 k + 3), read at every tile's
+  // phase re-seed from shared memory instead of the parameter space
+  unsigned long long* f_s = reinterpret_cast<unsigned long long*>(code_s + C::kCodeBytes + 16);
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());           // which half of the groups
@@ -186,6 +190,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
   for (int i = tid; i < C::kBins / 4; i += C::kThreads)
     reinterpret_cast<float4*>(bins)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tid < 3 * kHeads) mslot[tid] = ord_of(-INFINITY);
+  if (tid < 4 * kLocalGroups) f_s[tid] = a.phase.F[4 * rank * kLocalGroups + tid];
 
   // queries of the 4 heads for this lane's 4 pairs, scaled so that scores are in log2
   // units.  Slot j holds head (k ^ j) & 3: with this lane-dependent order the butterfly
@@ -308,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<R>::kThreads, Cf
     float* pxb = peer_xchg + buf * (kTile * kHeads);
 
 #pragma unroll
-    for (int p = 0; p < 4; ++p) ph[p] = phase_at(a.phase.F[4 * G + (p ^ (2 * fk))], t_tile + sigma);
+    for (int p = 0; p < 4; ++p) ph[p] = phase_at(f_s[4 * k + (p ^ (2 * fk))], t_tile + sigma);
     float s_part[C::kSteps];
     constexpr int kGS = C::kSteps >= 4 ? 4 : C::kSteps;   // steps per pass group
 #pragma unroll

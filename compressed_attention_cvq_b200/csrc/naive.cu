@@ -25,6 +25,11 @@ __global__ void __launch_bounds__(kDqThreads) naive_dequant_kernel(
     const uint8_t* __restrict__ val_codes, const int32_t* __restrict__ seq_lens, int R,
     int n_kv_heads, int t_cap, PhaseTurns phase, __half* __restrict__ k_out,
     __half* __restrict__ v_out) {
+  // F_j from shared memory: the 16 groups of a warp read 16 different pairs, and an indexed
+  // read of the parameter space serializes over distinct addresses
+  __shared__ unsigned long long f_tab[kPairs];
+  for (int i = threadIdx.x; i < kPairs; i += kDqThreads) f_tab[i] = phase.F[i];
+  __syncthreads();
   const int G = threadIdx.x & 15;
   const int t = blockIdx.x * (kDqThreads / 16) + (threadIdx.x >> 4);
   const int h = blockIdx.y, b = blockIdx.z;
@@ -53,7 +58,7 @@ __global__ void __launch_bounds__(kDqThreads) naive_dequant_kernel(
   __half2 ko[4], vo[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const float2 ph = phase_at(phase.F[4 * G + p], t);
+    const float2 ph = phase_at(f_tab[4 * G + p], t);
     ko[p] = __floats2half2_rn(ph.x * kr[p] - ph.y * ki[p], ph.y * kr[p] + ph.x * ki[p]);
     vo[p] = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
   }
@@ -72,6 +77,9 @@ __global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
     const uint8_t* __restrict__ val_codes, const int32_t* __restrict__ seq_lens, int R,
     int n_kv_heads, int t_cap, PhaseTurns phase, __half* __restrict__ k_out,
     __half* __restrict__ v_out, bool packed6) {
+  __shared__ unsigned long long f_tab[kPairs];      // F_j, as in naive_dequant_kernel
+  for (int i = threadIdx.y * 32 + threadIdx.x; i < kPairs; i += 256) f_tab[i] = phase.F[i];
+  __syncthreads();
   const int t = blockIdx.x * 32 + threadIdx.x;
   const int chunk = threadIdx.y;
   const int G = blockIdx.y & 1, h = blockIdx.y >> 1, b = blockIdx.z;
@@ -103,7 +111,7 @@ __global__ void __launch_bounds__(256) naive_dequant_wide_kernel(
   __half2 ko[4], vo[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const float2 ph = phase_at(phase.F[kWidePairs * G + 4 * chunk + p], t);
+    const float2 ph = phase_at(f_tab[kWidePairs * G + 4 * chunk + p], t);
     ko[p] = __floats2half2_rn(ph.x * k[2 * p] - ph.y * k[2 * p + 1],
                               ph.y * k[2 * p] + ph.x * k[2 * p + 1]);
     vo[p] = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
