@@ -63,8 +63,8 @@ constexpr size_t kRedBytes = sizeof(float) * (2 * kWWarps * kWHeads + 4 * kWHead
 constexpr size_t kWSmem = kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kTCodeBytes + kRedBytes;
 static_assert(kWSteps * kWSlots == kWTile, "tile must be a whole number of steps");
 static_assert(kWSmem <= 227 * 1024, "shared memory per CTA");
-// the reduction region holds red_m, red_l, mref_s, l_s, fac_s and, in its last 16 bytes, the
-// 8-byte mbarrier of the codebook copies
+// the reduction region holds red_m, red_l, mref_s, l_s, 16 unused bytes and, in its last 16
+// bytes, the 8-byte mbarrier of the codebook copies
 static_assert(kRedBytes >= sizeof(float) * (2 * kWWarps * kWHeads + 3 * kWHeads) + 8, "mbarrier room");
 static_assert((kCwBytes + kBinBytes + kXchgBytes + kCodeBytes + kTCodeBytes +
                sizeof(float) * (2 * kWWarps * kWHeads + 3 * kWHeads)) % 8 == 0, "mbarrier alignment");
@@ -109,8 +109,7 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
   float* red_l = red_m + kWWarps * kWHeads;                                   // [16][4]
   float* mref_s = red_l + kWWarps * kWHeads;                                  // [4]
   float* l_s = mref_s + kWHeads;                                              // [4]
-  float* fac_s = l_s + kWHeads;                                               // [4] spare
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(fac_s + kWHeads);           // codebook copies
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(l_s + 2 * kWHeads);         // codebook copies
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
