@@ -31,7 +31,9 @@
 //   codes: [buffer][key | value][rc][256 tokens] bytes, copied with cp.async from the
 //     planar global layout [B, Hkv, 2, R, t_cap] while the previous tile computes, then
 //     transposed once per tile to [key | value][256 tokens][16 bytes] so a token's rc codes
-//     come in one 16-byte load.
+//     come in one 16-byte load; a token's value bytes are stored rotated to the round order
+//     of its bin updates (its token slot's starting round first), so the update loop reads
+//     byte i at a position fixed at compile time.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -199,16 +201,15 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
   }
   // queries, scaled to log2 units; slot j holds head (k ^ j) & 3 (select-free reduction)
   const float qscale = kLog2e * 0.08838834764831845f;
-  float qv[kWHeads][4][2];
+  float2 qv[kWHeads][4];                 // (real, imaginary) of pair p for head slot j
 #pragma unroll
   for (int j = 0; j < kWHeads; ++j) {
     const int hh = (k ^ j) & 3;
     const size_t qrow = (static_cast<size_t>(b) * a.n_q_heads + hq0 + hh) * kHeadDim;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      qv[j][p][0] = load_q(a.q, a.q_dtype, qrow + 2 * jp[p]) * qscale;
-      qv[j][p][1] = load_q(a.q, a.q_dtype, qrow + 2 * jp[p] + 1) * qscale;
-    }
+    for (int p = 0; p < 4; ++p)
+      qv[j][p] = make_float2(load_q(a.q, a.q_dtype, qrow + 2 * jp[p]) * qscale,
+                             load_q(a.q, a.q_dtype, qrow + 2 * jp[p] + 1) * qscale);
   }
 
   const int n_tiles = (t_end - t_begin + kWTile - 1) / kWTile;
@@ -237,6 +238,19 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
                                      : static_cast<uint32_t>(src[r * kWTile]);
           wv[r >> 2] |= c << (8 * (r & 3));
         }
+      if (kind == 1) {
+        // value codes in the order the token's bin updates take them: byte i = round
+        // (rf + i) mod rc, rf = the round its token slot starts at (token t & 7 mod rc)
+        const int rf = (t & 7) % rc;
+        const unsigned __int128 v = (static_cast<unsigned __int128>(wv[2]) << 64) |
+                                    (static_cast<unsigned __int128>(wv[1]) << 32) | wv[0];
+        const unsigned __int128 mask = (static_cast<unsigned __int128>(1) << (8 * rc)) - 1;
+        const unsigned __int128 rot =
+            rf == 0 ? v : (((v >> (8 * rf)) | (v << (8 * (rc - rf)))) & mask);
+        wv[0] = static_cast<uint32_t>(rot);
+        wv[1] = static_cast<uint32_t>(rot >> 32);
+        wv[2] = static_cast<uint32_t>(rot >> 64);
+      }
       *reinterpret_cast<uint4*>(tcode + (kind * kWTile + t) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     __syncthreads();
@@ -268,15 +282,18 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
           }
         }
       }
-      float P[kWHeads] = {0.f, 0.f, 0.f, 0.f};
+      // rotate each pair, project on the 4 heads with packed (real, imaginary) FMAs
+      float2 P2[kWHeads];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float xr = acc[p].x, xi = acc[p].y;
-        const float zr = fmaf(ph[p].x, xr, -ph[p].y * xi);
-        const float zi = fmaf(ph[p].x, xi, ph[p].y * xr);
+        const float2 z = make_float2(fmaf(ph[p].x, xr, -ph[p].y * xi), fmaf(ph[p].x, xi, ph[p].y * xr));
 #pragma unroll
-        for (int j = 0; j < kWHeads; ++j) P[j] = fmaf(qv[j][p][0], zr, fmaf(qv[j][p][1], zi, P[j]));
+        for (int j = 0; j < kWHeads; ++j) P2[j] = p == 0 ? __fmul2_rn(qv[j][p], z) : __ffma2_rn(qv[j][p], z, P2[j]);
       }
+      float P[kWHeads];
+#pragma unroll
+      for (int j = 0; j < kWHeads; ++j) P[j] = P2[j].x + P2[j].y;
       // sum over the token's 8 lanes; lane k ends with head k & 3
       const float s0 = P[0] + __shfl_xor_sync(0xffffffffu, P[2], 2);
       const float s1 = P[1] + __shfl_xor_sync(0xffffffffu, P[3], 2);
@@ -345,8 +362,9 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
 #pragma unroll
       for (int i = 0; i < kRC; ++i) {
         if (i < rc) {
-          const uint32_t wd = r < 4 ? v4.x : (r < 8 ? v4.y : v4.z);
-          const int c = (wd >> (8 * (r & 3))) & (kWideCodes - 1);
+          // byte i holds round r = (r_first + i) mod rc (rotated in the transpose)
+          const uint32_t wd = i < 4 ? v4.x : (i < 8 ? v4.y : v4.z);
+          const int c = (wd >> (8 * (i & 3))) & (kWideCodes - 1);
           if (in_bounds(a.fault, c * kBinStride + 4 * r + hh, kWideCodes * kBinStride))
             atomicAdd(&bins[c * kBinStride + 4 * r + hh], wt);
           r = (r + 1 == rc) ? 0 : r + 1;
