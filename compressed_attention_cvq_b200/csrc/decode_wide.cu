@@ -260,7 +260,9 @@ __device__ __forceinline__ void wide_body(const DecodeArgs& a, int R) {
     float2 ph[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) ph[p] = phase_at(F[p], t_tile + tt0);
-#pragma unroll 1
+    // four steps unrolled: the next token's codeword loads are issued while the previous
+    // token's rotation, projection and shuffle reduction complete
+#pragma unroll 4
     for (int step = 0; step < kWSteps; ++step) {
       const int tt = step * kWSlots + tt0;
       float2 acc[4];
