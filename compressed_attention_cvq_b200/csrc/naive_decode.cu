@@ -1,9 +1,10 @@
 // Decode attention over the fp16 keys / values written by naive_dequant_kernel (the naive
 // path's second half).  One CTA per (split, KV head, sequence) for its NG query heads.
-// 8 lanes per token, each lane 16 dims (one 32-byte load of K and of V); the partial dot
-// products are summed over the 8 lanes with shuffles; every 8-lane group keeps its own
+// 16 lanes per token, each lane 8 dims (one 16-byte load of K and of V); the partial dot
+// products are summed over the 16 lanes with shuffles; every 16-lane group keeps its own
 // online-softmax state for its token stream, merged across streams in shared memory at
-// the end.  m is the exact split maximum.
+// the end.  m is the exact split maximum.  With 8 dims per lane the 4-head kernel holds
+// its queries and accumulators in ~100 registers, so two CTAs fit an SM.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -12,11 +13,13 @@ namespace cvq {
 
 namespace {
 
-constexpr int kNvThreads = 256;                 // 8 warps x 4 token streams
-constexpr int kStreams = kNvThreads / 8;        // 32 token streams per CTA
+constexpr int kNvThreads = 256;                 // 8 warps x 2 token streams
+constexpr int kLanesPerToken = 16;
+constexpr int kDimsPerLane = kHeadDim / kLanesPerToken;   // 8
+constexpr int kStreams = kNvThreads / kLanesPerToken;     // 16 token streams per CTA
 
 template <int NG>
-__global__ void __launch_bounds__(kNvThreads) naive_decode_kernel(
+__global__ void __launch_bounds__(kNvThreads, 2) naive_decode_kernel(
     const void* __restrict__ q, int q_dtype, const __half* __restrict__ kc,
     const __half* __restrict__ vc, const int32_t* __restrict__ seq_lens, int n_q_heads,
     int n_kv_heads, int t_cap, int n_splits, int split_tokens, float* __restrict__ part_o,
@@ -24,8 +27,8 @@ __global__ void __launch_bounds__(kNvThreads) naive_decode_kernel(
   extern __shared__ float sm[];                 // [kStreams][NG][128 + 2]
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31;
-  const int stream = tid >> 3;                  // token stream (8 lanes each)
-  const int k = lane & 7;                       // dims 16k .. 16k + 15
+  const int stream = tid / kLanesPerToken;      // token stream (16 lanes each)
+  const int k = lane % kLanesPerToken;          // dims 8k .. 8k + 7
   const int hq0 = h * NG;
   int L = seq_lens[b];
   L = L < 0 ? 0 : (L > t_cap ? t_cap : L);
@@ -34,55 +37,54 @@ __global__ void __launch_bounds__(kNvThreads) naive_decode_kernel(
   const size_t part_row = (static_cast<size_t>(b) * n_q_heads + hq0) * n_splits + split;
 
   const float qscale = kLog2e * 0.08838834764831845f;
-  float qv[NG][16];
+  float qv[NG][kDimsPerLane];
 #pragma unroll
   for (int hh = 0; hh < NG; ++hh) {
 #pragma unroll
-    for (int d = 0; d < 16; ++d)
-      qv[hh][d] = load_q(q, q_dtype, (static_cast<size_t>(b) * n_q_heads + hq0 + hh) * kHeadDim + 16 * k + d) * qscale;
+    for (int d = 0; d < kDimsPerLane; ++d)
+      qv[hh][d] = load_q(q, q_dtype, (static_cast<size_t>(b) * n_q_heads + hq0 + hh) * kHeadDim +
+                                         kDimsPerLane * k + d) * qscale;
   }
-  float m[NG], l[NG], o[NG][16];
+  float m[NG], l[NG], o[NG][kDimsPerLane];
 #pragma unroll
   for (int hh = 0; hh < NG; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
 #pragma unroll
-    for (int d = 0; d < 16; ++d) o[hh][d] = 0.f;
+    for (int d = 0; d < kDimsPerLane; ++d) o[hh][d] = 0.f;
   }
   const size_t row0 = (static_cast<size_t>(b) * n_kv_heads + h) * t_cap;
-  // the 8 lanes of a stream run the same number of iterations, but the streams of one warp
+  // the 16 lanes of a stream run the same number of iterations, but the streams of one warp
   // may not (tail of the split): shuffles name only the stream's own lanes
-  const unsigned gmask = 0xffu << (lane & 24);
+  const unsigned gmask = 0xffffu << (lane & 16);
   for (int t = t_begin + stream; t < t_end; t += kStreams) {
-    const uint4* kp = reinterpret_cast<const uint4*>(kc + (row0 + t) * kHeadDim + 16 * k);
-    const uint4* vp = reinterpret_cast<const uint4*>(vc + (row0 + t) * kHeadDim + 16 * k);
-    const uint4 k0 = __ldg(kp), k1 = __ldg(kp + 1), v0 = __ldg(vp), v1 = __ldg(vp + 1);
+    const uint4 k0 = __ldg(reinterpret_cast<const uint4*>(kc + (row0 + t) * kHeadDim + kDimsPerLane * k));
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(vc + (row0 + t) * kHeadDim + kDimsPerLane * k));
     const __half2* kh0 = reinterpret_cast<const __half2*>(&k0);
-    const __half2* kh1 = reinterpret_cast<const __half2*>(&k1);
     const __half2* vh0 = reinterpret_cast<const __half2*>(&v0);
-    const __half2* vh1 = reinterpret_cast<const __half2*>(&v1);
-    float kf[16], vf[16];
+    float kf[kDimsPerLane], vf[kDimsPerLane];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 a = __half22float2(kh0[i]), c = __half22float2(kh1[i]);
-      kf[2 * i] = a.x; kf[2 * i + 1] = a.y; kf[8 + 2 * i] = c.x; kf[8 + 2 * i + 1] = c.y;
-      a = __half22float2(vh0[i]); c = __half22float2(vh1[i]);
-      vf[2 * i] = a.x; vf[2 * i + 1] = a.y; vf[8 + 2 * i] = c.x; vf[8 + 2 * i + 1] = c.y;
+      float2 a = __half22float2(kh0[i]);
+      kf[2 * i] = a.x; kf[2 * i + 1] = a.y;
+      a = __half22float2(vh0[i]);
+      vf[2 * i] = a.x; vf[2 * i + 1] = a.y;
     }
 #pragma unroll
     for (int hh = 0; hh < NG; ++hh) {
       float s = 0.f;
 #pragma unroll
-      for (int d = 0; d < 16; ++d) s = fmaf(qv[hh][d], kf[d], s);
+      for (int d = 0; d < kDimsPerLane; ++d) s = fmaf(qv[hh][d], kf[d], s);
       s += __shfl_xor_sync(gmask, s, 1);
       s += __shfl_xor_sync(gmask, s, 2);
       s += __shfl_xor_sync(gmask, s, 4);
+      s += __shfl_xor_sync(gmask, s, 8);
       const float m_new = fmaxf(m[hh], s);
       const float f = exp2f(m[hh] - m_new);   // 0 on the first token (m = -inf)
       const float w = exp2f(s - m_new);
       l[hh] = l[hh] * f + w;
 #pragma unroll
-      for (int d = 0; d < 16; ++d) o[hh][d] = fmaf(o[hh][d], f, w * vf[d]);
+      for (int d = 0; d < kDimsPerLane; ++d) o[hh][d] = fmaf(o[hh][d], f, w * vf[d]);
       m[hh] = m_new;
     }
   }
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(kNvThreads) naive_decode_kernel(
 #pragma unroll
   for (int hh = 0; hh < NG; ++hh) {
 #pragma unroll
-    for (int d = 0; d < 16; ++d) st[hh * (kHeadDim + 2) + 16 * k + d] = o[hh][d];
+    for (int d = 0; d < kDimsPerLane; ++d) st[hh * (kHeadDim + 2) + kDimsPerLane * k + d] = o[hh][d];
     if (k == 0) {
       st[hh * (kHeadDim + 2) + kHeadDim] = m[hh];
       st[hh * (kHeadDim + 2) + kHeadDim + 1] = l[hh];
