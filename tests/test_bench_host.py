@@ -127,6 +127,6 @@ def _python_sources():
 @pytest.mark.parametrize("rel", _python_sources())
 def test_every_global_name_resolves(rel):
     """A function that reads a name its module never binds (a missing import) fails only
-    when that function runs, on the GPU machine for most of these files: check statically."""
+    when that function runs, on a GPU machine for most of these files: check statically."""
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     assert _unresolved_globals(os.path.join(root, rel)) == []
