@@ -49,6 +49,8 @@ def _ptxas_report(src):
     ("decode_gqa.cu", "decode_gqa4_kernelILi1E", 128),
     ("decode_gqa.cu", "decode_gqa4_kernelILi2E", 128),
     ("decode_wide.cu", "decode_wide_kernel", 128),
+    # the naive attention's 4-head instance runs two 256-thread CTAs per SM
+    ("naive_decode.cu", "naive_decode_kernelILi4E", 128),
 ])
 def test_decode_kernels_fit_their_register_budget(src, kernel, max_regs):
     res = _ptxas_report(os.path.join(ROOT, "compressed_attention_cvq_b200", "csrc", src))
