@@ -85,12 +85,13 @@ typedef enum {
 typedef enum { CVQ_F32 = 0, CVQ_BF16 = 1 } cvq_dtype;
 
 typedef struct {
-  int32_t batch;      /* B  >= 1                                              */
-  int32_t n_q_heads;  /* Hq >= 1, a multiple of n_kv_heads                   */
+  int32_t batch;      /* 1 <= B <= 65535                                      */
+  int32_t n_q_heads;  /* 1 <= Hq <= 65535, a multiple of n_kv_heads          */
   int32_t n_kv_heads; /* Hkv >= 1; Hq/Hkv in {1, 2, 4, 8}                     */
   int32_t head_dim;   /* must be 128                                          */
   int32_t R;          /* residual rounds: 1 or 2 (g = 8), 1..22 (g = 64)      */
-  int32_t t_cap;      /* token capacity of the code buffers per sequence, >= 0 */
+  int32_t t_cap;      /* token capacity of the code buffers per sequence, >= 0
+                         (group_dim 64: a multiple of 16)                      */
   float rope_base;    /* RoPE base, > 1 (500000 for LLaMA-3.1)                */
   int32_t group_dim;  /* scalars per quantization group: 0 or 8 (default), 64 */
   int32_t code_bits;  /* storage of a code: 0 or 8 = one byte per code (default);

@@ -3,6 +3,7 @@ entry point include/cvq.h declares, reports sizes, and rejects bad arguments wit
 status before launching anything.  Every call below carries at least one invalid
 argument or has nothing to do (t_cap = 0), so none of them reaches a kernel launch."""
 import ctypes
+import math
 import os
 import re
 
@@ -355,3 +356,47 @@ def test_c_attend_loop_compiles(tmp_path):
         pytest.skip(str(e))
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 1 and "usage" in r.stderr
+
+
+def _valid_by_header(b, hq, hkv, hd, R, t_cap, base, gd, cb):
+    """The shape rules cvq.h states for cvq_shape, restated."""
+    if hd != 128 or gd not in (0, 8, 64) or cb not in (0, 8, 6):
+        return False
+    if gd == 64:
+        if not 1 <= R <= 22 or t_cap % 16 != 0 or (cb == 6 and t_cap % 64 != 0):
+            return False
+    elif R not in (1, 2) or cb == 6:
+        return False
+    if not (1 <= b <= 65535 and 1 <= hq <= 65535 and hkv >= 1 and t_cap >= 0):
+        return False
+    if hq % hkv != 0 or hq // hkv not in (1, 2, 4, 8):
+        return False
+    return math.isfinite(base) and base > 1.0
+
+
+def test_shape_rules_match_the_header():
+    """Random shapes, many of them invalid in one field: the library accepts exactly the
+    shapes the header's rules accept (cvq_partials_bytes > 0), and then sizes the partial
+    states as B x Hq x n_splits x 130 floats."""
+    import random
+
+    b_ = b
+    rng = random.Random(12345)
+    pick = lambda *xs: xs[rng.randrange(len(xs))]
+    for _ in range(4000):
+        bb = pick(1, 2, 7, 0, -1, 65535, 65536)
+        hkv = pick(1, 2, 3, 8, 0)
+        hq = pick(hkv, 2 * hkv, 4 * hkv, 8 * hkv, 3 * hkv, 16 * hkv, hkv + 1, 0, 70000)
+        hd = pick(128, 128, 128, 64)
+        R = pick(1, 2, 3, 11, 21, 22, 23, 0)
+        gd = pick(0, 8, 64, 64, 16)
+        cb = pick(0, 8, 6, 6, 4)
+        t_cap = pick(0, 64, 100, 96, 4096, 131072, -1)
+        base = pick(500000.0, 10000.0, 1.0, 0.5, float("inf"), float("nan"))
+        s = b_.make_shape(bb, hq, hkv, R, t_cap, base, head_dim=hd, group_dim=gd, code_bits=cb)
+        n = rng.randrange(1, 40)
+        got = b_.lib.cvq_partials_bytes(ctypes.byref(s), n)
+        ok = _valid_by_header(bb, hq, hkv, hd, R, t_cap, base, gd, cb)
+        assert (got > 0) == ok, (bb, hq, hkv, hd, R, t_cap, base, gd, cb, got)
+        if ok:
+            assert got == bb * hq * n * 130 * 4
